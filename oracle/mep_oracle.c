@@ -1,0 +1,289 @@
+/*
+ * CPU oracle for MoonEP's balanced expert-parallel token plan and its data
+ * movement.  TEST INFRASTRUCTURE ONLY: the product path never links, loads or
+ * calls this file; only the test suite, the smoke check and the CPU-baseline
+ * leg of the benchmark do.  It shares no code, header, table or helper with
+ * the CUDA library, and includes nothing from it.
+ *
+ * Plain, single-threaded C99 (built with -O2 -ffp-contract=off, no SIMD
+ * intrinsics, no threads).  Floating-point results are accumulated in binary64
+ * and rounded once at the end; integer results are the plain definitions.
+ *
+ * Sources, by page title and section:
+ *   [P1-why]  "Moonshot AI Open-Sources MoonEP, the Library Used to Train the
+ *             MoE Model Kimi K3", section "Why expert parallelism is needed":
+ *             the router sends each token to its top-K experts; skew metric
+ *             maxvio = max_e(T_e / T-bar) - 1, zero meaning perfect balance.
+ *   [P2-prob] "Moonshot AI Open-Sources MoonEP: A Perfectly Balanced Expert
+ *             Parallelism Library for MoE Training", section "The problem
+ *             MoonEP targets": T_e is the number of tokens routed to expert e,
+ *             T-bar the count expected under perfect balance.
+ *   [P1-how]  first title, section "How MoonEP works": every rank receives
+ *             exactly S x K tokens; a few redundant experts are scheduled
+ *             online from the current router output; their gradients are
+ *             reduced back to the home ranks on the backward pass.
+ *   [P1-eng]  first title, section "Why this matters to engineers": static
+ *             buffer shapes, zero-copy, tokens written straight into
+ *             positions grouped by expert; section "Key facts": B = E/R for
+ *             training.
+ *
+ * Readings where the pages are silent (each is also listed in the design
+ * notes): T-bar = R*S*K/E; the schedule is the stable sort of all (token, k)
+ * pairs by (expert, global token g = r*S + s, k) cut into R contiguous chunks
+ * of S*K slots; home(e) = e / (E/R); a (rank, expert) segment whose rank is
+ * not home(e) is a replica; combine is the K-term weighted sum back to token
+ * order; the replica reduction sums an expert's segment rows in ascending
+ * segment order.
+ */
+#include <math.h>
+#include <stddef.h>
+#include <stdint.h>
+#include <string.h>
+
+#define ORA_OK 0
+#define ORA_ERR_ARG 1
+#define ORA_ERR_DATA 2
+
+/* ---- bf16 <-> binary32 / binary64, from the IEEE 754 layouts ----------- */
+
+/* A bf16 value is the upper half of the binary32 with the same sign,
+ * exponent and leading seven fraction bits. */
+float ora_bf16_to_f32(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+/* Round a binary64 value to the nearest bf16, ties to even significand.
+ * bf16: 1 sign bit, 8 exponent bits (bias 127), 7 stored fraction bits.
+ * Normal binade [2^q, 2^(q+1)) has spacing 2^(q-7); below 2^-126 the spacing
+ * stays 2^-133 (subnormals).  Overflow past the largest finite value plus
+ * half a spacing gives infinity. */
+uint16_t ora_f64_to_bf16(double d)
+{
+    uint16_t sign = signbit(d) ? 0x8000u : 0u;
+    if (isnan(d))
+        return (uint16_t)(sign | 0x7FC0u);
+    double a = fabs(d);
+    if (isinf(a))
+        return (uint16_t)(sign | 0x7F80u);
+    if (a == 0.0)
+        return sign;
+    int ex;
+    (void)frexp(a, &ex);              /* a in [2^(ex-1), 2^ex) */
+    int q = ex - 1;                   /* binade exponent */
+    if (q < -126)
+        q = -126;                     /* subnormal spacing */
+    double spacing = ldexp(1.0, q - 7);
+    double t = a / spacing;           /* exact: division by a power of two */
+    double n = floor(t);
+    double rem = t - n;               /* exact */
+    if (rem > 0.5 || (rem == 0.5 && fmod(n, 2.0) != 0.0))
+        n += 1.0;
+    double v = n * spacing;           /* exact, representable in bf16 */
+    /* largest finite bf16 = (2^8 - 1) * 2^120 */
+    if (v > ldexp(255.0, 120))
+        return (uint16_t)(sign | 0x7F80u);
+    float f = (float)v;               /* exact */
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    return (uint16_t)(sign | ((u >> 16) & 0x7FFFu));
+}
+
+/* ---- shape rules -------------------------------------------------------- */
+
+static int ora_check_shape(int R, int S, int E, int K)
+{
+    if (R < 1 || S < 1 || E < 1 || K < 1 || K > E)
+        return ORA_ERR_ARG;
+    if (E % R != 0)                   /* home(e) = e / (E/R) needs E/R whole */
+        return ORA_ERR_ARG;
+    if ((int64_t)R * S * K > INT32_MAX)
+        return ORA_ERR_ARG;
+    return ORA_OK;
+}
+
+/* ---- T_e and maxvio  [P1-why], [P2-prob] -------------------------------- */
+
+/* counts[e] = T_e = number of (token, k) pairs routed to expert e. */
+int ora_counts(int R, int S, int E, int K, const int32_t *idx, int32_t *counts)
+{
+    int st = ora_check_shape(R, S, E, K);
+    if (st)
+        return st;
+    int64_t NK = (int64_t)R * S * K;
+    for (int e = 0; e < E; ++e)
+        counts[e] = 0;
+    for (int64_t p = 0; p < NK; ++p) {
+        int32_t e = idx[p];
+        if (e < 0 || e >= E)
+            return ORA_ERR_DATA;
+        counts[e] += 1;
+    }
+    return ORA_OK;
+}
+
+/* maxvio = max_e T_e / T-bar - 1 with T-bar = R*S*K/E, written as one
+ * binary64 quotient of two exact integers: (max T_e * E) / (R*S*K) - 1. */
+double ora_maxvio_from_counts(int R, int S, int E, int K, const int32_t *counts,
+                              int32_t *max_count)
+{
+    int32_t m = 0;
+    for (int e = 0; e < E; ++e)
+        if (counts[e] > m)
+            m = counts[e];
+    if (max_count)
+        *max_count = m;
+    int64_t NK = (int64_t)R * S * K;
+    return (double)((int64_t)m * E) / (double)NK - 1.0;
+}
+
+/* ---- the plan  [P1-how], [P1-eng] --------------------------------------- *
+ * Output arrays (caller-allocated):
+ *   counts[E], expert_offset[E+1], slot[N*K], src_pair[N*K],
+ *   seg[4*(E+R-1)] as {expert, rank, start, count},
+ *   rank_seg_ptr[R+1], expert_seg_ptr[E+1], replica_seg[E+R-1],
+ *   num_seg, num_replicas, max_count (scalars), maxvio.
+ */
+int ora_plan(int R, int S, int E, int K, const int32_t *idx,
+             int32_t *counts, int32_t *expert_offset, int32_t *slot,
+             int32_t *src_pair, int32_t *seg, int32_t *num_seg,
+             int32_t *num_replicas, int32_t *rank_seg_ptr,
+             int32_t *expert_seg_ptr, int32_t *replica_seg,
+             int32_t *max_count, double *maxvio)
+{
+    int st = ora_counts(R, S, E, K, idx, counts);
+    if (st)
+        return st;
+    int64_t N = (int64_t)R * S;
+    int64_t SK = (int64_t)S * K;
+    int64_t NK = N * K;
+    int B = E / R;                            /* home experts per rank */
+
+    *maxvio = ora_maxvio_from_counts(R, S, E, K, counts, max_count);
+
+    /* Expert e's slots start after all pairs of experts e' < e. */
+    expert_offset[0] = 0;
+    for (int e = 0; e < E; ++e)
+        expert_offset[e + 1] = expert_offset[e] + counts[e];
+
+    /* Stable counting sort: visit pairs in (g, k) order; each takes the next
+     * free slot of its expert.  This is the sort by (expert, g, k). */
+    for (int e = 0; e < E; ++e)
+        counts[e] = 0;                        /* reused as per-expert cursor */
+    for (int64_t g = 0; g < N; ++g) {
+        for (int k = 0; k < K; ++k) {
+            int64_t pair = g * K + k;
+            int32_t e = idx[pair];
+            int32_t p = expert_offset[e] + counts[e];
+            counts[e] += 1;
+            slot[pair] = p;
+            src_pair[p] = (int32_t)pair;
+        }
+    }
+    /* counts[] is the histogram again after the walk. */
+
+    /* Cut the slot range into R chunks of S*K; a segment is a maximal run of
+     * slots with the same (rank, expert). */
+    int32_t ns = 0;
+    int32_t prev_r = -1, prev_e = -1;
+    for (int64_t p = 0; p < NK; ++p) {
+        int32_t e = idx[src_pair[p]];
+        int32_t r = (int32_t)(p / SK);
+        if (r != prev_r || e != prev_e) {
+            seg[4 * ns + 0] = e;
+            seg[4 * ns + 1] = r;
+            seg[4 * ns + 2] = (int32_t)(p - (int64_t)r * SK);
+            seg[4 * ns + 3] = 0;
+            ns += 1;
+            prev_r = r;
+            prev_e = e;
+        }
+        seg[4 * (ns - 1) + 3] += 1;
+    }
+    *num_seg = ns;
+
+    /* A segment hosted away from its expert's home rank is a replica. */
+    int32_t nr = 0;
+    for (int32_t s = 0; s < ns; ++s) {
+        int32_t e = seg[4 * s + 0], r = seg[4 * s + 1];
+        if (r != e / B)
+            replica_seg[nr++] = s;
+    }
+    *num_replicas = nr;
+
+    /* CSR pointers: first segment on rank >= r, first segment of expert >= e. */
+    int32_t s = 0;
+    for (int r = 0; r <= R; ++r) {
+        while (s < ns && seg[4 * s + 1] < r)
+            ++s;
+        rank_seg_ptr[r] = s;
+    }
+    s = 0;
+    for (int e = 0; e <= E; ++e) {
+        while (s < ns && seg[4 * s + 0] < e)
+            ++s;
+        expert_seg_ptr[e] = s;
+    }
+    return ORA_OK;
+}
+
+/* ---- zero-copy dispatch  [P1-eng] --------------------------------------- *
+ * buf[p, :] = x[src_pair[p] / K, :] for the nslots slots listed. */
+void ora_dispatch(int64_t nslots, int K, int64_t H, const int32_t *src_pair,
+                  const uint16_t *x, uint16_t *buf)
+{
+    for (int64_t p = 0; p < nslots; ++p) {
+        int64_t g = src_pair[p] / K;
+        memcpy(buf + p * H, x + g * H, (size_t)H * sizeof(uint16_t));
+    }
+}
+
+/* ---- weighted combine back to token order -------------------------------- *
+ * out[g, h] = sum_k w[g,k] * y[slot[g,k], h], summed in binary64 and rounded
+ * once to bf16.  exact[] (may be NULL) receives the binary64 sum and absum[]
+ * (may be NULL) the sum of |w * y| terms, for error bounds. */
+void ora_combine(int64_t ntok, int K, int64_t H, const int32_t *slot,
+                 const float *w, const uint16_t *y, uint16_t *out,
+                 double *exact, double *absum)
+{
+    for (int64_t g = 0; g < ntok; ++g) {
+        for (int64_t h = 0; h < H; ++h) {
+            double acc = 0.0, mag = 0.0;
+            for (int k = 0; k < K; ++k) {
+                int64_t p = slot[g * K + k];
+                double term = (double)w[g * K + k] * (double)ora_bf16_to_f32(y[p * H + h]);
+                acc += term;
+                mag += fabs(term);
+            }
+            out[g * H + h] = ora_f64_to_bf16(acc);
+            if (exact)
+                exact[g * H + h] = acc;
+            if (absum)
+                absum[g * H + h] = mag;
+        }
+    }
+}
+
+/* ---- replica weight-gradient reduction  [P1-how] ------------------------ *
+ * home[e, i] = sum over expert e's segments s (ascending) of G[s, i], zero
+ * for an expert with no segment.  G has one row of P floats per segment. */
+void ora_reduce(int E, const int32_t *expert_seg_ptr, int64_t P,
+                const float *G, double *home, double *absum)
+{
+    for (int e = 0; e < E; ++e) {
+        for (int64_t i = 0; i < P; ++i) {
+            double acc = 0.0, mag = 0.0;
+            for (int32_t s = expert_seg_ptr[e]; s < expert_seg_ptr[e + 1]; ++s) {
+                double v = (double)G[(int64_t)s * P + i];
+                acc += v;
+                mag += fabs(v);
+            }
+            home[(int64_t)e * P + i] = acc;
+            if (absum)
+                absum[(int64_t)e * P + i] = mag;
+        }
+    }
+}
