@@ -1,0 +1,420 @@
+#!/usr/bin/env python
+"""Throughput of the balanced expert-parallel hot path on B200.
+
+One step = one pass of the whole path over one batch of synthetic input:
+mep_plan (T_e, maxvio, offsets, stable scatter, segments, replicas) ->
+mep_dispatch -> mep_combine -> mep_reduce_replica_grads, all through the C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mep|reference]
+
+* value: tokens per second of the whole job (tokens of all ranks / max-over-ranks
+  device time), inputs resident in HBM, L2 flushed (512 MB write) between
+  steps outside the timed events.
+* e2e: the same metric through the public API with pinned host buffers: every
+  step copies that step's inputs host->device and the outputs back.
+* roofline: the step's dominant kernel, algorithmic bytes / its mean event
+  time, against the measured HBM copy peak.
+* cpu_baseline / --impl reference: the CPU oracle, single-threaded, on a
+  bounded sample of the same workload, scaled to tokens per second.
+Multi-GPU (torchrun): every rank runs an independent replica of the
+single-device problem ("replicas only"); timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "plan+dispatch+combine tokens/sec and HBM GB/s (% of roofline), 1 B200"
+FALLBACK_HBM_GBS = 6650.0
+FLUSH_BYTES = 512 << 20
+KERNEL_SOURCES = {"plan": "plan.cu", "dispatch": "dispatch.cu", "combine": "combine.cu",
+                  "reduce": "reduce.cu"}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["mep", "reference"], default="mep")
+    ap.add_argument("--workload", default=workloads.BENCH_WORKLOAD,
+                    choices=list(workloads.WORKLOADS))
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="target CPU time of the oracle baseline sample")
+    return ap.parse_args()
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_sha(name: str) -> str:
+    p = os.path.join(ROOT, "token_dispatch_mep_b200", "csrc", KERNEL_SOURCES[name])
+    with open(p, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:12]
+
+
+def dram_traffic(name: str, workload: str):
+    """Per-launch DRAM bytes of `name` on `workload` from the committed ncu
+    summary, or None if absent or taken on a different kernel source."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    sha = kernel_sha(name)
+    with open(path) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) >= 4 and not line.startswith("#") and parts[0] == name \
+                    and parts[1] == workload and parts[3] == sha:
+                return float(parts[2])
+    return None
+
+
+# ------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples the SM clock and the clock-event reasons with NVML every
+    ~20 ms in a background thread (reads only; changes no setting)."""
+
+    BITS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+            0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, device_index: int):
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._h = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            try:
+                props = torch.cuda.get_device_properties(device_index)
+                bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+                self._h = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+            except Exception:
+                self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self._nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._h = None
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        nv = self._nv
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = get_reasons(self._h)
+                for bit, name in self.BITS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.02)
+
+    def start(self):
+        if self._h is not None:
+            self._t.start()
+        return self
+
+    def stop(self):
+        self._stop.set()
+        if self._h is not None:
+            self._t.join()
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------ CPU oracle leg
+
+def oracle_throughput(wl, target_seconds: float, host=None):
+    """Time the oracle, as it stands, on a bounded sample of the workload:
+    the whole plan, dispatch and combine of the first n tokens, the reduction
+    of the first c gradient columns; scaled to tokens per second of the full
+    step.  Single-threaded C."""
+    import oracle
+    ora = oracle.get()
+    R, S, E, K, H, P, N = wl.R, wl.S, wl.E, wl.K, wl.H, wl.P, wl.N
+    if host is None:
+        idx, w = workloads.routing(wl)
+        host = dict(idx=idx, w=w)
+    idx, w = host["idx"], host["w"]
+    t0 = time.perf_counter()
+    pl = ora.plan(R, S, E, K, idx)
+    t_plan = time.perf_counter() - t0
+    # size the samples from the budget (about 12 ns per combine term, 3 ns per
+    # reduced element on this kind of host core)
+    per_tok = K * H * 12.5e-9
+    n_tok = int(max(1, min(N, (0.5 * target_seconds) / per_tok)))
+    x = workloads.hidden(n_tok, H, seed=1).view(__import__("torch").int16).numpy().view(np.uint16)
+    y = workloads.expert_outputs(n_tok * K, H, seed=2).view(__import__("torch").int16).numpy().view(np.uint16)
+    pairs = np.arange(n_tok * K, dtype=np.int32)
+    t0 = time.perf_counter()
+    ora.dispatch(K, pairs, x)
+    t_disp = time.perf_counter() - t0
+    local_slot = np.arange(n_tok * K, dtype=np.int32).reshape(n_tok, K)
+    t0 = time.perf_counter()
+    ora.combine(local_slot, w[:n_tok], y)
+    t_comb = time.perf_counter() - t0
+    t_red, n_col = 0.0, 0
+    if P:
+        n_col = int(max(1, min(P, (0.4 * target_seconds) / (3.2e-9 * (wl.seg_rows + E)))))
+        G = workloads.seg_grads(wl.seg_rows, n_col, seed=3).numpy()
+        t0 = time.perf_counter()
+        ora.reduce(pl["expert_seg_ptr"], G)
+        t_red = time.perf_counter() - t0
+    t_step = t_plan + (t_disp + t_comb) * (N / n_tok) + (t_red * (P / n_col) if P else 0.0)
+    sample = (f"whole plan; dispatch+combine of {n_tok}/{N} tokens; "
+              f"reduce of {n_col}/{P} gradient columns; scaled to the full step")
+    return dict(value=N / t_step, t_step=t_step, sample=sample,
+                measured_s=t_plan + t_disp + t_comb + t_red,
+                parts=dict(plan=t_plan, dispatch=t_disp, combine=t_comb, reduce=t_red))
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    wl = workloads.WORKLOADS[args.workload]
+    idx, w = workloads.routing(wl)
+    host = dict(idx=idx, w=w)
+    budget = max(0.5, min(4.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_throughput(wl, budget, host)
+    vals = [oracle_throughput(wl, budget, host) for _ in range(max(1, args.steps))]
+    t = statistics.mean(v["t_step"] for v in vals)
+    value = wl.N / t
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": t * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "R": wl.R, "S": wl.S, "E": wl.E, "K": wl.K,
+                   "H": wl.H, "P": wl.P},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": vals[0]["sample"]},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# -------------------------------------------------------------- GPU arm
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    import torch
+    import torch.distributed as dist
+
+    import token_dispatch_mep_b200 as mep
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    wl = workloads.WORKLOADS[args.workload]
+    R, S, E, K, H, P, N, NK = wl.R, wl.S, wl.E, wl.K, wl.H, wl.P, wl.N, wl.NK
+    s = mep.Shape(R, S, E, K)
+    idx_h, w_h = workloads.routing(wl, seed=0)
+    idx = torch.from_numpy(idx_h).to(dev)
+    w = torch.from_numpy(w_h).to(dev)
+    x = workloads.hidden(N, H, seed=1, device=dev)
+    y = workloads.expert_outputs(NK, H, seed=2, device=dev)
+    G = workloads.seg_grads(wl.seg_rows, P, seed=3, device=dev) if P else None
+    plan = mep.Plan(s, dev)
+    buf = torch.empty((R, S * K, H), dtype=torch.bfloat16, device=dev)
+    out = torch.empty((N, H), dtype=torch.bfloat16, device=dev)
+    home = torch.empty((E, P), dtype=torch.float32, device=dev) if P else None
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step(evs=None):
+        if evs:
+            evs[0].record()
+        mep.mep_plan(s, idx, plan)
+        if evs:
+            evs[1].record()
+        mep.mep_dispatch(s, H, plan, x, buf)
+        if evs:
+            evs[2].record()
+        mep.mep_combine(s, H, plan, y, w, out)
+        if evs:
+            evs[3].record()
+        if P:
+            mep.mep_reduce_replica_grads(s, plan, P, G, home)
+        if evs:
+            evs[4].record()
+
+    launches_per_step = 4 if P else 3
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if mep.mep_read_status(plan) != 0:
+        raise RuntimeError("device status not OK after warm-up")
+    num_seg = plan.host()["num_seg"]
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    sampler = ClockSampler(local).start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        step(evs[i])
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    st = mep.mep_read_status(plan)
+    if st != 0:
+        raise RuntimeError(f"device status {mep.mep_status_string(st)}")
+
+    stage = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)]
+                      for i in range(args.steps)])          # ms
+    ms_step = float(stage.sum(axis=1).mean())
+    if world > 1:
+        t = torch.tensor([ms_step], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_step = float(t.item())
+    value = N * world / (ms_step * 1e-3)
+
+    stage_ms = dict(zip(["plan", "dispatch", "combine", "reduce"], stage.mean(axis=0).tolist()))
+    algo = {
+        "plan": 3 * NK * 4,
+        "dispatch": N * H * 2 + NK * H * 2 + NK * 4,
+        "combine": NK * H * 2 + NK * 4 + NK * 4 + N * H * 2,
+        "reduce": (num_seg + E) * P * 4,
+    }
+    peak, peak_kind = measured_peak()
+    kernels = {}
+    for k in ("plan", "dispatch", "combine", "reduce"):
+        if k == "reduce" and not P:
+            continue
+        gbs = algo[k] / (stage_ms[k] * 1e-3) / 1e9
+        kernels[k] = {"ms": stage_ms[k], "bytes": algo[k], "gbs": gbs, "frac": gbs / peak}
+    dom = max((k for k in kernels if k != "plan"), key=lambda k: kernels[k]["ms"])
+    roofline = {"bound": "hbm", "achieved": kernels[dom]["gbs"], "peak": peak, "unit": "GB/s",
+                "frac": kernels[dom]["gbs"] / peak, "traffic": dram_traffic(dom, wl.name),
+                "kernel": dom, "peak_source": f"{peak_kind} hbm_gbs (copy)"}
+
+    # ---- e2e: host buffers through the public API
+    e2e = None
+    if args.e2e_steps > 0:
+        pin = dict(pin_memory=True)
+        hi = torch.from_numpy(idx_h).pin_memory()
+        hw = torch.from_numpy(w_h).pin_memory()
+        hx = torch.empty(x.shape, dtype=x.dtype, **pin).copy_(x)
+        hy = torch.empty(y.shape, dtype=y.dtype, **pin).copy_(y)
+        hG = torch.empty(G.shape, dtype=G.dtype, **pin).copy_(G) if P else None
+        ho = torch.empty(out.shape, dtype=out.dtype, **pin)
+        hh = torch.empty(home.shape, dtype=home.dtype, **pin) if P else None
+        hsc = torch.empty(4, dtype=torch.int32, **pin)
+        hmv = torch.empty(1, dtype=torch.float64, **pin)
+        h2d = sum(t.numel() * t.element_size() for t in (hi, hw, hx, hy) + ((hG,) if P else ()))
+        d2h = sum(t.numel() * t.element_size() for t in (ho, hsc, hmv) + ((hh,) if P else ()))
+
+        def e2e_step():
+            idx.copy_(hi, non_blocking=True)
+            w.copy_(hw, non_blocking=True)
+            x.copy_(hx, non_blocking=True)
+            y.copy_(hy, non_blocking=True)
+            if P:
+                G.copy_(hG, non_blocking=True)
+            step()
+            ho.copy_(out, non_blocking=True)
+            if P:
+                hh.copy_(home, non_blocking=True)
+            hsc.copy_(plan.scalars, non_blocking=True)
+            hmv.copy_(plan.maxvio_t, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e1.record()
+        torch.cuda.synchronize()
+        ms_e2e = e0.elapsed_time(e1) / args.e2e_steps
+        if world > 1:
+            t = torch.tensor([ms_e2e], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms_e2e = float(t.item())
+        if int(hsc[3].item()) != 0:
+            raise RuntimeError("device status not OK after e2e steps")
+        e2e = {"value": N * world / (ms_e2e * 1e-3), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        r = oracle_throughput(wl, args.cpu_seconds, dict(idx=idx_h, w=w_h))
+        cpu = {"value": r["value"], "unit": "tokens/s", "cores": 1, "kind": "oracle",
+               "sample": r["sample"], "measured_s": r["measured_s"]}
+
+    if rank == 0:
+        pdc_ms = stage_ms["plan"] + stage_ms["dispatch"] + stage_ms["combine"]
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": wl.name, "R": R, "S": S, "E": E, "K": K, "H": H, "P": P,
+                       "step": "plan+dispatch+combine+replica-grad reduce",
+                       "l2": "flushed by a 512 MB write between steps, outside the events",
+                       "parallelism": f"replicas x{world}"},
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "clocks": clocks,
+            "gpu_launches": launches_per_step * args.steps,
+            "stages_ms": stage_ms,
+            "kernels": kernels,
+            "plan_us": stage_ms["plan"] * 1e3,
+            "pdc_tokens_per_s": N * world / (pdc_ms * 1e-3),
+            "num_seg": num_seg,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,203 @@
+/*
+ * mep.h -- C ABI of libmep: MoonEP's balanced expert-parallel token plan and
+ * its data movement, as hand-written CUDA kernels for one B200 (sm_100a).
+ *
+ * What the library computes (sources named by page title and section):
+ *
+ *   "Moonshot AI Open-Sources MoonEP, the Library Used to Train the MoE Model
+ *   Kimi K3" (below: the MoonEP release page)
+ *     - "Why expert parallelism is needed": the router sends every token to
+ *       its top-K experts; skew is measured as maxvio = max_e(T_e / T-bar) - 1,
+ *       zero being perfect balance.
+ *     - "How MoonEP works": every EP rank receives exactly S x K tokens however
+ *       skewed the routing; a small number of redundant experts are scheduled
+ *       online from the current router output; their gradients are reduced
+ *       back to the home ranks on the backward pass.
+ *     - "Why this matters to engineers": static buffer shapes and zero-copy --
+ *       tokens are written straight into positions grouped by expert, with no
+ *       per-layer host synchronisation.
+ *   "Moonshot AI Open-Sources MoonEP: A Perfectly Balanced Expert Parallelism
+ *   Library for MoE Training", "The problem MoonEP targets": T_e counts the
+ *   tokens routed to expert e; T-bar is the count expected under perfect
+ *   balance.
+ *
+ * The pages give no scheduling algorithm.  This library fixes one: the stable
+ * sort of all (token, k) pairs by (expert, global token g, k), cut into R
+ * contiguous chunks of S*K slots.  Chunk r is rank r's static receive buffer;
+ * a (rank, expert) run inside it is a segment; a segment on a rank other
+ * than home(e) = e / (E/R) hosts a replica of expert e.
+ *
+ * Notation.  R simulated ranks, S tokens per rank, E experts, K experts per
+ * token, H hidden size.  N = R*S tokens, global token g = r*S + s (rank-major),
+ * pair (g, k) has flat index g*K + k, NK = N*K pairs = slots, SK = S*K slots per
+ * rank, global slot p in [0, NK), rank(p) = p / SK.
+ *
+ * Conventions for every call.
+ *   - All buffers are caller-owned device memory; the library never allocates
+ *     or frees.  Scratch comes from a caller-supplied workspace.
+ *   - Every call is asynchronous and stream-ordered on `stream` (a
+ *     cudaStream_t; NULL is the legacy default stream).  No call synchronises
+ *     the host except mep_read_status.
+ *   - Host-detected errors (bad shape, NULL or misaligned pointer, small
+ *     workspace) return immediately and launch nothing.
+ *   - Device-detected errors (an expert id outside [0, E), a slot or segment
+ *     pointer outside its range, a wait that timed out) are written into the
+ *     plan's device status word; the first error wins.  Outputs are undefined
+ *     when the status is not MEP_OK, but no kernel ever reads or writes
+ *     outside the buffers described here.
+ *   - bf16 buffers are typed uint16_t (raw bf16 bit patterns) so that C callers
+ *     need no CUDA headers.
+ *   - The current CUDA device is the one the buffers live on.
+ */
+#ifndef MEP_H
+#define MEP_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define MEP_API __attribute__((visibility("default")))
+#else
+#define MEP_API
+#endif
+
+#define MEP_VERSION 1
+#define MEP_MAX_EXPERTS 1024      /* E <= 1024 */
+#define MEP_MAX_RANKS 1024        /* R <= 1024 */
+#define MEP_MAX_HIDDEN 32768      /* H <= 32768 bf16 elements per row */
+#define MEP_MAX_TOPK 16           /* K <= 16 */
+
+typedef enum {
+    MEP_OK = 0,
+    MEP_ERR_INVALID_ARG = 1,  /* shape rule broken or NULL pointer */
+    MEP_ERR_MISALIGNED = 2,   /* row buffers need 16-byte alignment and H % 8 == 0 */
+    MEP_ERR_WORKSPACE = 3,    /* workspace NULL, not 256-byte aligned, or too small */
+    MEP_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed */
+    MEP_ERR_DEVICE_DATA = 5,  /* device saw an expert id / slot / segment pointer out of range */
+    MEP_ERR_TIMEOUT = 6       /* a bounded device-side wait ran out */
+} mep_status_t;
+
+/* Shape rules: R, S, E, K >= 1; K <= E; K <= MEP_MAX_TOPK; E % R == 0
+ * (home(e) = e / (E/R)); E <= MEP_MAX_EXPERTS; R <= MEP_MAX_RANKS;
+ * R*S*K < 2^31. */
+typedef struct {
+    int32_t R, S, E, K;
+} mep_shape_t;
+
+/* One (rank, expert) run of slots: slots [rank*SK + start, rank*SK + start +
+ * count) all hold pairs routed to `expert`.  16 bytes. */
+typedef struct {
+    int32_t expert, rank, start, count;
+} mep_segment_t;
+
+/* The plan: device pointers, caller-owned, sized from the shape alone.
+ * Segments are ordered by slot, which is also (rank, expert) order and
+ * (expert, rank) order; at most E + R - 1 exist. */
+typedef struct {
+    int32_t *counts;          /* [E]     T_e                                    */
+    int32_t *expert_offset;   /* [E+1]   first slot of expert e; [E] = NK        */
+    int32_t *slot;            /* [N*K]   pair (g,k) -> global slot p             */
+    int32_t *src_pair;        /* [N*K]   slot p -> pair index g*K + k            */
+    mep_segment_t *seg;       /* [E+R-1] segments in slot order                  */
+    int32_t *rank_seg_ptr;    /* [R+1]   rank r owns segments [ptr[r], ptr[r+1]) */
+    int32_t *expert_seg_ptr;  /* [E+1]   expert e owns segments [ptr[e], ptr[e+1]) */
+    int32_t *replica_seg;     /* [E+R-1] indices of replica segments, ascending  */
+    int32_t *num_seg;         /* [1]                                             */
+    int32_t *num_replicas;    /* [1]     segments with rank != home(expert)      */
+    int32_t *max_count;       /* [1]     max_e T_e                               */
+    int32_t *status;          /* [1]     device error word (mep_status_t)        */
+    double *maxvio;           /* [1]     max_e(T_e / T-bar) - 1, T-bar = NK / E  */
+} mep_plan_t;
+
+/* Bytes of workspace mep_plan and mep_maxvio need for this shape.  The
+ * workspace must be zero-filled once before its first use (e.g. by
+ * cudaMemsetAsync); every call that returns MEP_OK and ends with device
+ * status MEP_OK leaves it ready for the next call.  After MEP_ERR_TIMEOUT or
+ * MEP_ERR_CUDA, zero it again.  One workspace serves one stream at a time. */
+MEP_API size_t mep_plan_workspace_bytes(mep_shape_t shape);
+
+/* T_e and maxvio only ("Why expert parallelism is needed", release page).
+ *   topk_idx  int32 [N, K] row-major, expert ids of each token's top-K.
+ *   counts    int32 [E] out: T_e.
+ *   max_count int32 [1] out: max_e T_e.
+ *   maxvio    double [1] out: (double)(max_count * E) / (double)(N*K) - 1.0,
+ *             one IEEE binary64 division of two exact integers.
+ *   status    int32 [1] out: device error word, cleared by this call.
+ *   ws        workspace of mep_plan_workspace_bytes(shape) bytes, 256-byte aligned. */
+MEP_API mep_status_t mep_maxvio(mep_shape_t shape, const int32_t *topk_idx,
+                        int32_t *counts, int32_t *max_count, double *maxvio,
+                        int32_t *status, void *ws, size_t ws_bytes, void *stream);
+
+/* The balanced plan ("How MoonEP works"; "Why this matters to engineers").
+ *   topk_idx  int32 [N, K] row-major.
+ *   plan      every field written: counts, maxvio and max_count as in
+ *             mep_maxvio; expert_offset = exclusive prefix sum of counts;
+ *             slot[g*K+k] = expert_offset[e] + #{(g',k') before (g,k) in
+ *             (g, k) order with the same expert e}; src_pair its inverse;
+ *             the segments, CSR pointers and replica list of the R-way cut.
+ *             plan->status is cleared at the start of the call.
+ * Each rank r receives exactly SK slots, [r*SK, (r+1)*SK), grouped by expert. */
+MEP_API mep_status_t mep_plan(mep_shape_t shape, const int32_t *topk_idx,
+                      const mep_plan_t *plan, void *ws, size_t ws_bytes,
+                      void *stream);
+
+/* Zero-copy dispatch into the static receive buffer ("Why this matters to
+ * engineers": tokens written straight into positions grouped by expert).
+ *   x    bf16 [N, H], 16-byte aligned; H % 8 == 0, 8 <= H <= MEP_MAX_HIDDEN.
+ *   buf  bf16 [R, S*K, H] out, 16-byte aligned: buf[slot[g,k], :] = x[g, :]
+ *        for every pair; a token routed to several experts is copied once
+ *        per slot.  Bit-exact copies. */
+MEP_API mep_status_t mep_dispatch(mep_shape_t shape, int32_t H, const mep_plan_t *plan,
+                          const uint16_t *x, uint16_t *buf, void *stream);
+
+/* Weighted combine back to token order (the return leg of the top-K routing
+ * in "Why expert parallelism is needed").
+ *   y      bf16 [R, S*K, H] expert outputs in slot order, 16-byte aligned.
+ *   topk_w float32 [N, K] router weights.
+ *   out    bf16 [N, H] out: out[g,:] = bf16_rne(sum over k = 0..K-1, in that
+ *          order, of w[g,k] * y[slot[g,k], :]), accumulated in float32 with a
+ *          fused multiply-add per term. */
+MEP_API mep_status_t mep_combine(mep_shape_t shape, int32_t H, const mep_plan_t *plan,
+                         const uint16_t *y, const float *topk_w, uint16_t *out,
+                         void *stream);
+
+/* Backward reduction of replica weight-gradients into their home expert
+ * ("How MoonEP works": gradients reduced back to the home ranks).
+ *   seg_grads  float32 [E+R-1, P]: row s is the gradient computed by segment
+ *              s of the plan (its rank's copy of expert seg[s].expert); rows
+ *              s >= num_seg are ignored.  16-byte aligned when P % 4 == 0.
+ *   home_grads float32 [E, P] out: home_grads[e,:] = sum of rows
+ *              expert_seg_ptr[e] .. expert_seg_ptr[e+1]-1, ascending, in
+ *              float32; zero for an expert with no segment.
+ *   P >= 0; P == 0 is a no-op. */
+MEP_API mep_status_t mep_reduce_replica_grads(mep_shape_t shape, const mep_plan_t *plan,
+                                      int64_t P, const float *seg_grads,
+                                      float *home_grads, void *stream);
+
+/* Synchronises `stream` and returns the plan's device status word (MEP_OK if
+ * every call so far on this plan ran clean), or MEP_ERR_CUDA if the copy
+ * itself fails.  The only call that blocks the host. */
+MEP_API mep_status_t mep_read_status(const mep_plan_t *plan, void *stream);
+
+/* Static, human-readable name of a status code. */
+MEP_API const char *mep_status_string(mep_status_t status);
+
+/* Upper bound, in nanoseconds of the GPU global timer, on every device-side
+ * wait (grid barriers in the plan, transfer barriers in dispatch).  A wait
+ * that runs out records MEP_ERR_TIMEOUT and the kernel returns.  Process-wide;
+ * default 1e9 (one second); values below 1000 are raised to 1000. */
+MEP_API void mep_set_wait_limit_ns(uint64_t ns);
+MEP_API uint64_t mep_get_wait_limit_ns(void);
+
+/* MEP_VERSION of the built library. */
+MEP_API int32_t mep_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MEP_H */

@@ -1,0 +1,124 @@
+"""The C-ABI library builds, loads and exports every symbol include/mep.h
+declares; host-side argument checks reject bad calls before any CUDA call.
+CPU only: no kernel is launched here."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import token_dispatch_mep_b200 as mep
+from token_dispatch_mep_b200 import build as mep_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    mep_build.build()
+    return mep.load_library()
+
+
+def header_symbols():
+    names = set()
+    for f in os.listdir(os.path.join(ROOT, "include")):
+        if f.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", f)).read()
+            names |= set(re.findall(r"MEP_API\s+[^;(]*?\b(mep_\w+)\s*\(", text))
+    return names
+
+
+def test_header_declares_the_calls():
+    names = header_symbols()
+    for n in ("mep_maxvio", "mep_plan", "mep_dispatch", "mep_combine",
+              "mep_reduce_replica_grads", "mep_plan_workspace_bytes", "mep_read_status"):
+        assert n in names
+    assert names == set(mep.ABI_SYMBOLS)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    raw = ctypes.CDLL(mep.library_path())
+    for n in header_symbols():
+        assert hasattr(raw, n), n
+
+
+def test_version_and_strings(lib):
+    assert mep.mep_version() == 1
+    for code, name in mep.STATUS.items():
+        assert mep.mep_status_string(code)
+    assert mep.mep_status_string(99) == "unknown status"
+
+
+def test_wait_limit_roundtrip(lib):
+    old = mep.mep_get_wait_limit_ns()
+    try:
+        mep.mep_set_wait_limit_ns(5_000_000)
+        assert mep.mep_get_wait_limit_ns() == 5_000_000
+        mep.mep_set_wait_limit_ns(3)
+        assert mep.mep_get_wait_limit_ns() == 1000
+    finally:
+        mep.mep_set_wait_limit_ns(old)
+
+
+def test_workspace_bytes(lib):
+    S = mep.Shape
+    assert mep.mep_plan_workspace_bytes(S(8, 4096, 64, 6)) >= 64 * 4
+    assert mep.mep_plan_workspace_bytes(S(2, 2, 3, 2)) == 0          # E % R != 0
+    assert mep.mep_plan_workspace_bytes(S(1, 1, 2048, 1)) == 0       # E > 1024
+    assert mep.mep_plan_workspace_bytes(S(1, 4, 32, 17)) == 0        # K > 16
+    assert mep.mep_plan_workspace_bytes(S(1 << 10, 1 << 20, 1024, 16)) == 0  # R*S*K >= 2^31
+    a = mep.mep_plan_workspace_bytes(S(64, 2048, 896, 16))
+    b = mep.mep_plan_workspace_bytes(S(64, 8, 896, 16))
+    assert a == b  # sized from E alone: static across token counts
+
+
+def _plan_struct(base=0x10000):
+    p = mep._PlanStruct()
+    for i, (name, _) in enumerate(mep._PlanStruct._fields_):
+        setattr(p, name, base + 256 * i)
+    return p
+
+
+def test_host_side_rejections_launch_nothing(lib):
+    L = lib
+    s = mep.Shape(2, 4, 4, 2)
+    vp = ctypes.c_void_p
+    good = vp(0x100000)
+    p = _plan_struct()
+    # bad shapes
+    for bad in [mep.Shape(0, 4, 4, 2), mep.Shape(2, 4, 3, 2), mep.Shape(2, 4, 4, 5),
+                mep.Shape(2, -1, 4, 2), mep.Shape(2, 4, 4, 0)]:
+        assert L.mep_plan(bad, good, ctypes.byref(p), good, 1 << 30, None) == 1
+        assert L.mep_dispatch(bad, 8, ctypes.byref(p), good, good, None) == 1
+    # NULL pointers
+    assert L.mep_plan(s, None, ctypes.byref(p), good, 1 << 30, None) == 1
+    assert L.mep_plan(s, good, None, good, 1 << 30, None) == 1
+    assert L.mep_dispatch(s, 8, ctypes.byref(p), None, good, None) == 1
+    assert L.mep_combine(s, 8, ctypes.byref(p), good, None, good, None) == 1
+    assert L.mep_reduce_replica_grads(s, ctypes.byref(p), 16, None, good, None) == 1
+    assert L.mep_reduce_replica_grads(s, ctypes.byref(p), -1, good, good, None) == 1
+    assert L.mep_reduce_replica_grads(s, ctypes.byref(p), 0, None, None, None) == 0  # no-op
+    # misalignment and hidden-size rules
+    assert L.mep_dispatch(s, 8, ctypes.byref(p), vp(0x100002), good, None) == 2
+    assert L.mep_dispatch(s, 12, ctypes.byref(p), good, good, None) == 2
+    assert L.mep_dispatch(s, 4, ctypes.byref(p), good, good, None) == 1
+    assert L.mep_dispatch(s, 65536, ctypes.byref(p), good, good, None) == 1
+    assert L.mep_combine(s, 8, ctypes.byref(p), good, vp(0x100002), good, None) == 2
+    assert L.mep_reduce_replica_grads(s, ctypes.byref(p), 16, vp(0x100004), good, None) == 2
+    q = _plan_struct()
+    q.seg = 0x100008
+    assert L.mep_plan(s, good, ctypes.byref(q), good, 1 << 30, None) == 2
+    # workspace rules
+    assert L.mep_plan(s, good, ctypes.byref(p), None, 1 << 30, None) == 3
+    assert L.mep_plan(s, good, ctypes.byref(p), vp(0x100080), 1 << 30, None) == 3
+    assert L.mep_plan(s, good, ctypes.byref(p), good, 16, None) == 3
+    i4 = vp(0x100000)
+    assert L.mep_maxvio(s, i4, i4, i4, vp(0x100004), i4, good, 1 << 30, None) == 2
+    assert L.mep_maxvio(s, i4, i4, i4, good, i4, good, 8, None) == 3
+
+
+def test_package_has_no_cpu_fallback(tmp_path, monkeypatch):
+    monkeypatch.setattr(mep, "_lib", None)
+    monkeypatch.setattr(mep, "_LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError):
+        mep.load_library()

@@ -1,0 +1,273 @@
+"""Python binding of libmep, MoonEP's balanced expert-parallel token plan and
+its data movement as CUDA kernels for B200 (sm_100a).
+
+Argument marshalling only: every step runs in the CUDA kernels behind the C
+ABI declared in ``include/mep.h``; PyTorch supplies device memory and
+streams.  The functions carry the C names (``mep_plan``, ``mep_dispatch``,
+...) and take torch tensors; they check dtypes, devices and sizes (the C ABI
+cannot see sizes), pass raw pointers and the current stream, and raise
+``MepError`` on a non-zero status.  There is no CPU fallback: without the
+built library every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "MepError", "Shape", "Plan", "load_library", "library_path",
+    "mep_plan_workspace_bytes", "mep_maxvio", "mep_plan", "mep_dispatch", "mep_combine",
+    "mep_reduce_replica_grads", "mep_read_status", "mep_status_string",
+    "mep_set_wait_limit_ns", "mep_get_wait_limit_ns", "mep_version", "STATUS",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libmep.so")
+
+STATUS = {0: "MEP_OK", 1: "MEP_ERR_INVALID_ARG", 2: "MEP_ERR_MISALIGNED", 3: "MEP_ERR_WORKSPACE",
+          4: "MEP_ERR_CUDA", 5: "MEP_ERR_DEVICE_DATA", 6: "MEP_ERR_TIMEOUT"}
+
+# Symbols the header declares; the CPU test suite checks they are exported.
+ABI_SYMBOLS = ("mep_plan_workspace_bytes", "mep_maxvio", "mep_plan", "mep_dispatch", "mep_combine",
+               "mep_reduce_replica_grads", "mep_read_status", "mep_status_string",
+               "mep_set_wait_limit_ns", "mep_get_wait_limit_ns", "mep_version")
+
+
+class MepError(RuntimeError):
+    def __init__(self, code: int, where: str = ""):
+        self.code = int(code)
+        super().__init__(f"{where}: {STATUS.get(self.code, self.code)}")
+
+
+class Shape(ctypes.Structure):
+    """``mep_shape_t``: R ranks, S tokens per rank, E experts, K experts per token."""
+    _fields_ = [("R", ctypes.c_int32), ("S", ctypes.c_int32), ("E", ctypes.c_int32),
+                ("K", ctypes.c_int32)]
+
+    @property
+    def N(self) -> int:
+        return self.R * self.S
+
+    @property
+    def NK(self) -> int:
+        return self.R * self.S * self.K
+
+    @property
+    def SK(self) -> int:
+        return self.S * self.K
+
+    @property
+    def seg_rows(self) -> int:
+        return self.E + self.R - 1
+
+    def __repr__(self):
+        return f"Shape(R={self.R}, S={self.S}, E={self.E}, K={self.K})"
+
+
+class _PlanStruct(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "counts", "expert_offset", "slot", "src_pair", "seg", "rank_seg_ptr", "expert_seg_ptr",
+        "replica_seg", "num_seg", "num_replicas", "max_count", "status", "maxvio")]
+
+
+_lib = None
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load_library():
+    """Load ``libmep.so`` (built in-tree by ``token_dispatch_mep_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise RuntimeError(f"{_LIB_PATH} is missing: build it with "
+                           "`python -m token_dispatch_mep_b200.build` (nvcc, sm_100a)")
+    L = ctypes.CDLL(_LIB_PATH)
+    vp, i32, i64, u64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint64
+    sz = ctypes.c_size_t
+    P = ctypes.POINTER(_PlanStruct)
+    sig = {
+        "mep_plan_workspace_bytes": ([Shape], sz),
+        "mep_maxvio": ([Shape, vp, vp, vp, vp, vp, vp, sz, vp], ctypes.c_int),
+        "mep_plan": ([Shape, vp, P, vp, sz, vp], ctypes.c_int),
+        "mep_dispatch": ([Shape, i32, P, vp, vp, vp], ctypes.c_int),
+        "mep_combine": ([Shape, i32, P, vp, vp, vp, vp], ctypes.c_int),
+        "mep_reduce_replica_grads": ([Shape, P, i64, vp, vp, vp], ctypes.c_int),
+        "mep_read_status": ([P, vp], ctypes.c_int),
+        "mep_status_string": ([ctypes.c_int], ctypes.c_char_p),
+        "mep_set_wait_limit_ns": ([u64], None),
+        "mep_get_wait_limit_ns": ([], u64),
+        "mep_version": ([], i32),
+    }
+    for name, (args, res) in sig.items():
+        f = getattr(L, name)
+        f.argtypes = args
+        f.restype = res
+    _lib = L
+    return L
+
+
+def _shape(shape) -> Shape:
+    if isinstance(shape, Shape):
+        return shape
+    return Shape(*[int(v) for v in shape])
+
+
+def _stream(dev: torch.device):
+    return ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+
+
+def _need(t: torch.Tensor, name: str, dtype, numel: int, device: torch.device):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if t.device != device:
+        raise ValueError(f"{name}: on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.numel() < numel:
+        raise ValueError(f"{name}: {t.numel()} elements, need {numel}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _ok(code: int, where: str):
+    if code != 0:
+        raise MepError(code, where)
+
+
+class Plan:
+    """Device buffers of one plan (``mep_plan_t``), sized from the shape alone,
+    plus a zero-filled workspace for ``mep_plan`` / ``mep_maxvio``."""
+
+    def __init__(self, shape, device=None):
+        self.shape = _shape(shape)
+        s = self.shape
+        if device is None:
+            device = torch.device("cuda", torch.cuda.current_device())
+        self.device = torch.device(device)
+        i32 = dict(dtype=torch.int32, device=self.device)
+        self.counts = torch.zeros(s.E, **i32)
+        self.expert_offset = torch.zeros(s.E + 1, **i32)
+        self.slot = torch.zeros((s.N, s.K), **i32)
+        self.src_pair = torch.zeros(s.NK, **i32)
+        self.seg = torch.zeros((s.seg_rows, 4), **i32)
+        self.rank_seg_ptr = torch.zeros(s.R + 1, **i32)
+        self.expert_seg_ptr = torch.zeros(s.E + 1, **i32)
+        self.replica_seg = torch.zeros(s.seg_rows, **i32)
+        self.scalars = torch.zeros(4, **i32)  # num_seg, num_replicas, max_count, status
+        self.maxvio_t = torch.zeros(1, dtype=torch.float64, device=self.device)
+        nbytes = mep_plan_workspace_bytes(s)
+        if nbytes == 0:
+            raise MepError(1, "Plan")
+        self.workspace = torch.zeros(nbytes, dtype=torch.uint8, device=self.device)
+        a = lambda t: t.data_ptr()
+        sc = self.scalars.data_ptr()
+        self.struct = _PlanStruct(
+            a(self.counts), a(self.expert_offset), a(self.slot), a(self.src_pair), a(self.seg),
+            a(self.rank_seg_ptr), a(self.expert_seg_ptr), a(self.replica_seg),
+            sc, sc + 4, sc + 8, sc + 12, a(self.maxvio_t))
+
+    @property
+    def status_tensor(self) -> torch.Tensor:
+        return self.scalars[3:4]
+
+    def reset_workspace(self):
+        """Zero the workspace again (needed after MEP_ERR_TIMEOUT / MEP_ERR_CUDA)."""
+        self.workspace.zero_()
+
+    def host(self) -> dict:
+        """Copy every field to host numpy arrays (synchronises)."""
+        sc = self.scalars.cpu().tolist()
+        return dict(
+            counts=self.counts.cpu().numpy(), expert_offset=self.expert_offset.cpu().numpy(),
+            slot=self.slot.cpu().numpy(), src_pair=self.src_pair.cpu().numpy(),
+            seg=self.seg.cpu().numpy(), rank_seg_ptr=self.rank_seg_ptr.cpu().numpy(),
+            expert_seg_ptr=self.expert_seg_ptr.cpu().numpy(),
+            replica_seg=self.replica_seg.cpu().numpy(), num_seg=sc[0], num_replicas=sc[1],
+            max_count=sc[2], status=sc[3], maxvio=float(self.maxvio_t.item()))
+
+
+# ---------------------------------------------------------------- the calls
+
+def mep_plan_workspace_bytes(shape) -> int:
+    return int(load_library().mep_plan_workspace_bytes(_shape(shape)))
+
+
+def mep_maxvio(shape, topk_idx, counts, max_count, maxvio, status, workspace):
+    """T_e, max T_e and maxvio (device outputs)."""
+    L, s = load_library(), _shape(shape)
+    dev = topk_idx.device
+    args = [_need(topk_idx, "topk_idx", torch.int32, s.NK, dev),
+            _need(counts, "counts", torch.int32, s.E, dev),
+            _need(max_count, "max_count", torch.int32, 1, dev),
+            _need(maxvio, "maxvio", torch.float64, 1, dev),
+            _need(status, "status", torch.int32, 1, dev)]
+    ws = _need(workspace, "workspace", torch.uint8, mep_plan_workspace_bytes(s), dev)
+    _ok(L.mep_maxvio(s, *args, ws, workspace.numel(), _stream(dev)), "mep_maxvio")
+
+
+def mep_plan(shape, topk_idx, plan: Plan, workspace=None):
+    """The balanced plan of ``topk_idx`` (int32 [N, K]) into ``plan``."""
+    L, s = load_library(), _shape(shape)
+    dev = plan.device
+    idx = _need(topk_idx, "topk_idx", torch.int32, s.NK, dev)
+    ws_t = plan.workspace if workspace is None else workspace
+    ws = _need(ws_t, "workspace", torch.uint8, mep_plan_workspace_bytes(s), dev)
+    _ok(L.mep_plan(s, idx, ctypes.byref(plan.struct), ws, ws_t.numel(), _stream(dev)), "mep_plan")
+
+
+def mep_dispatch(shape, H: int, plan: Plan, x, buf):
+    """``buf[slot[g,k]] = x[g]``; x bf16 [N, H], buf bf16 [R, S*K, H]."""
+    L, s = load_library(), _shape(shape)
+    dev = plan.device
+    xp = _need(x, "x", torch.bfloat16, s.N * H, dev)
+    bp = _need(buf, "buf", torch.bfloat16, s.NK * H, dev)
+    _ok(L.mep_dispatch(s, int(H), ctypes.byref(plan.struct), xp, bp, _stream(dev)), "mep_dispatch")
+
+
+def mep_combine(shape, H: int, plan: Plan, y, topk_w, out):
+    """``out[g] = bf16(sum_k w[g,k] y[slot[g,k]])``; y bf16 [R, S*K, H], w fp32 [N, K]."""
+    L, s = load_library(), _shape(shape)
+    dev = plan.device
+    yp = _need(y, "y", torch.bfloat16, s.NK * H, dev)
+    wp = _need(topk_w, "topk_w", torch.float32, s.NK, dev)
+    op = _need(out, "out", torch.bfloat16, s.N * H, dev)
+    _ok(L.mep_combine(s, int(H), ctypes.byref(plan.struct), yp, wp, op, _stream(dev)), "mep_combine")
+
+
+def mep_reduce_replica_grads(shape, plan: Plan, P: int, seg_grads, home_grads):
+    """``home[e] = sum of seg_grads rows of e's segments``; seg_grads fp32
+    [E+R-1, P], home_grads fp32 [E, P]."""
+    L, s = load_library(), _shape(shape)
+    dev = plan.device
+    gp = _need(seg_grads, "seg_grads", torch.float32, s.seg_rows * P, dev)
+    hp = _need(home_grads, "home_grads", torch.float32, s.E * P, dev)
+    _ok(L.mep_reduce_replica_grads(s, ctypes.byref(plan.struct), int(P), gp, hp, _stream(dev)),
+        "mep_reduce_replica_grads")
+
+
+def mep_read_status(plan: Plan) -> int:
+    """Synchronise the current stream and return the plan's device status."""
+    return int(load_library().mep_read_status(ctypes.byref(plan.struct), _stream(plan.device)))
+
+
+def mep_status_string(code: int) -> str:
+    return load_library().mep_status_string(int(code)).decode()
+
+
+def mep_set_wait_limit_ns(ns: int):
+    load_library().mep_set_wait_limit_ns(int(ns))
+
+
+def mep_get_wait_limit_ns() -> int:
+    return int(load_library().mep_get_wait_limit_ns())
+
+
+def mep_version() -> int:
+    return int(load_library().mep_version())

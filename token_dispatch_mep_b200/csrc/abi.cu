@@ -1,0 +1,155 @@
+// The C ABI of libmep (declared in include/mep.h): argument checks, then one
+// kernel launch per call.  Nothing here allocates, frees or synchronises,
+// except mep_read_status.
+#include <atomic>
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+#include "mep.h"
+#include "mep_internal.h"
+
+namespace {
+
+std::atomic<uint64_t> g_wait_ns{1000000000ull};
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+mep_status_t check_shape(const mep_shape_t &s) {
+  if (s.R < 1 || s.S < 1 || s.E < 1 || s.K < 1) return MEP_ERR_INVALID_ARG;
+  if (s.K > s.E || s.K > MEP_MAX_TOPK) return MEP_ERR_INVALID_ARG;
+  if (s.E % s.R != 0) return MEP_ERR_INVALID_ARG;
+  if (s.E > MEP_MAX_EXPERTS || s.R > MEP_MAX_RANKS) return MEP_ERR_INVALID_ARG;
+  if ((int64_t)s.R * s.S * s.K > INT32_MAX) return MEP_ERR_INVALID_ARG;
+  return MEP_OK;
+}
+
+mep_status_t check_hidden(int32_t H) {
+  if (H < 8 || H > MEP_MAX_HIDDEN) return MEP_ERR_INVALID_ARG;
+  if (H % 8 != 0) return MEP_ERR_MISALIGNED;
+  return MEP_OK;
+}
+
+mep_status_t check_ws(const mep_shape_t &s, const void *ws, size_t ws_bytes) {
+  if (ws == nullptr || !aligned(ws, 256)) return MEP_ERR_WORKSPACE;
+  if (ws_bytes < mep::plan_workspace_bytes(s)) return MEP_ERR_WORKSPACE;
+  return MEP_OK;
+}
+
+mep_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? MEP_OK : MEP_ERR_CUDA; }
+
+cudaStream_t as_stream(void *s) { return static_cast<cudaStream_t>(s); }
+
+}  // namespace
+
+extern "C" {
+
+size_t mep_plan_workspace_bytes(mep_shape_t shape) {
+  if (check_shape(shape) != MEP_OK) return 0;
+  return mep::plan_workspace_bytes(shape);
+}
+
+mep_status_t mep_maxvio(mep_shape_t shape, const int32_t *topk_idx, int32_t *counts,
+                        int32_t *max_count, double *maxvio, int32_t *status, void *ws,
+                        size_t ws_bytes, void *stream) {
+  mep_status_t st = check_shape(shape);
+  if (st != MEP_OK) return st;
+  if (!topk_idx || !counts || !max_count || !maxvio || !status) return MEP_ERR_INVALID_ARG;
+  if (!aligned(topk_idx, 4) || !aligned(counts, 4) || !aligned(max_count, 4) ||
+      !aligned(status, 4) || !aligned(maxvio, 8))
+    return MEP_ERR_MISALIGNED;
+  if ((st = check_ws(shape, ws, ws_bytes)) != MEP_OK) return st;
+  mep_plan_t pl{};
+  pl.counts = counts;
+  pl.max_count = max_count;
+  pl.maxvio = maxvio;
+  pl.status = status;
+  return from_cuda(mep::launch_plan(shape, topk_idx, pl, 0, ws, g_wait_ns.load(), as_stream(stream)));
+}
+
+mep_status_t mep_plan(mep_shape_t shape, const int32_t *topk_idx, const mep_plan_t *plan, void *ws,
+                      size_t ws_bytes, void *stream) {
+  mep_status_t st = check_shape(shape);
+  if (st != MEP_OK) return st;
+  if (!topk_idx || !plan) return MEP_ERR_INVALID_ARG;
+  const mep_plan_t &p = *plan;
+  if (!p.counts || !p.expert_offset || !p.slot || !p.src_pair || !p.seg || !p.rank_seg_ptr ||
+      !p.expert_seg_ptr || !p.replica_seg || !p.num_seg || !p.num_replicas || !p.max_count ||
+      !p.status || !p.maxvio)
+    return MEP_ERR_INVALID_ARG;
+  const void *i32s[] = {topk_idx, p.counts, p.expert_offset, p.slot, p.src_pair, p.rank_seg_ptr,
+                        p.expert_seg_ptr, p.replica_seg, p.num_seg, p.num_replicas,
+                        p.max_count, p.status};
+  for (const void *q : i32s)
+    if (!aligned(q, 4)) return MEP_ERR_MISALIGNED;
+  if (!aligned(p.seg, 16) || !aligned(p.maxvio, 8)) return MEP_ERR_MISALIGNED;
+  if ((st = check_ws(shape, ws, ws_bytes)) != MEP_OK) return st;
+  return from_cuda(mep::launch_plan(shape, topk_idx, p, 1, ws, g_wait_ns.load(), as_stream(stream)));
+}
+
+mep_status_t mep_dispatch(mep_shape_t shape, int32_t H, const mep_plan_t *plan, const uint16_t *x,
+                          uint16_t *buf, void *stream) {
+  mep_status_t st = check_shape(shape);
+  if (st != MEP_OK) return st;
+  if ((st = check_hidden(H)) != MEP_OK) return st;
+  if (!plan || !plan->slot || !plan->status || !x || !buf) return MEP_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(buf, 16) || !aligned(plan->slot, 4)) return MEP_ERR_MISALIGNED;
+  return from_cuda(mep::launch_dispatch(shape, H, *plan, x, buf, g_wait_ns.load(), as_stream(stream)));
+}
+
+mep_status_t mep_combine(mep_shape_t shape, int32_t H, const mep_plan_t *plan, const uint16_t *y,
+                         const float *topk_w, uint16_t *out, void *stream) {
+  mep_status_t st = check_shape(shape);
+  if (st != MEP_OK) return st;
+  if ((st = check_hidden(H)) != MEP_OK) return st;
+  if (!plan || !plan->slot || !plan->status || !y || !topk_w || !out) return MEP_ERR_INVALID_ARG;
+  if (!aligned(y, 16) || !aligned(out, 16) || !aligned(topk_w, 4) || !aligned(plan->slot, 4))
+    return MEP_ERR_MISALIGNED;
+  return from_cuda(mep::launch_combine(shape, H, *plan, y, topk_w, out, as_stream(stream)));
+}
+
+mep_status_t mep_reduce_replica_grads(mep_shape_t shape, const mep_plan_t *plan, int64_t P,
+                                      const float *seg_grads, float *home_grads, void *stream) {
+  mep_status_t st = check_shape(shape);
+  if (st != MEP_OK) return st;
+  if (P < 0 || !plan) return MEP_ERR_INVALID_ARG;
+  if (P == 0) return MEP_OK;
+  if (!plan->expert_seg_ptr || !plan->status || !seg_grads || !home_grads)
+    return MEP_ERR_INVALID_ARG;
+  if ((int64_t)shape.E * P > ((int64_t)1 << 46)) return MEP_ERR_INVALID_ARG;
+  const size_t a = (P % 4 == 0) ? 16 : 4;
+  if (!aligned(seg_grads, a) || !aligned(home_grads, a) || !aligned(plan->expert_seg_ptr, 4))
+    return MEP_ERR_MISALIGNED;
+  return from_cuda(mep::launch_reduce(shape, *plan, P, seg_grads, home_grads, as_stream(stream)));
+}
+
+mep_status_t mep_read_status(const mep_plan_t *plan, void *stream) {
+  if (!plan || !plan->status) return MEP_ERR_INVALID_ARG;
+  int32_t host = 0;
+  cudaError_t e = cudaMemcpyAsync(&host, plan->status, sizeof host, cudaMemcpyDeviceToHost,
+                                  as_stream(stream));
+  if (e != cudaSuccess) return MEP_ERR_CUDA;
+  if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return MEP_ERR_CUDA;
+  return static_cast<mep_status_t>(host);
+}
+
+const char *mep_status_string(mep_status_t s) {
+  switch (s) {
+    case MEP_OK: return "ok";
+    case MEP_ERR_INVALID_ARG: return "invalid argument";
+    case MEP_ERR_MISALIGNED: return "misaligned pointer or hidden size";
+    case MEP_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case MEP_ERR_CUDA: return "CUDA error";
+    case MEP_ERR_DEVICE_DATA: return "out-of-range data seen on the device";
+    case MEP_ERR_TIMEOUT: return "device-side wait timed out";
+  }
+  return "unknown status";
+}
+
+void mep_set_wait_limit_ns(uint64_t ns) { g_wait_ns.store(ns < 1000 ? 1000 : ns); }
+
+uint64_t mep_get_wait_limit_ns(void) { return g_wait_ns.load(); }
+
+int32_t mep_version(void) { return MEP_VERSION; }
+
+}  // extern "C"

@@ -1,0 +1,35 @@
+// Internal launch entry points of libmep (host side, not part of the ABI).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+#include "mep.h"
+
+namespace mep {
+
+constexpr int kPlanThreads = 1024;
+constexpr int kPlanMaxBlocks = 1024;          // bound used to size the workspace
+constexpr int64_t kPlanMinPairsPerBlock = 4096;
+constexpr size_t kPlanWsHeader = 256;         // grid-barrier words
+
+size_t plan_workspace_bytes(const mep_shape_t &s);
+
+// full = 1: the whole plan; full = 0: counts, max_count, maxvio, status only.
+cudaError_t launch_plan(const mep_shape_t &s, const int32_t *idx, const mep_plan_t &pl,
+                        int full, void *ws, uint64_t wait_ns, cudaStream_t stream);
+
+cudaError_t launch_dispatch(const mep_shape_t &s, int32_t H, const mep_plan_t &pl,
+                            const uint16_t *x, uint16_t *buf, uint64_t wait_ns,
+                            cudaStream_t stream);
+
+cudaError_t launch_combine(const mep_shape_t &s, int32_t H, const mep_plan_t &pl,
+                           const uint16_t *y, const float *w, uint16_t *out,
+                           cudaStream_t stream);
+
+cudaError_t launch_reduce(const mep_shape_t &s, const mep_plan_t &pl, int64_t P,
+                          const float *G, float *home, cudaStream_t stream);
+
+}  // namespace mep

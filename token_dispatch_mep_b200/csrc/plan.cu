@@ -1,0 +1,362 @@
+// Plan kernel: T_e, maxvio, expert offsets, the stable counting-sort scatter
+// and the R-way cut into (rank, expert) segments, in one cooperative launch.
+//
+// The method (MoonEP release page "Moonshot AI Open-Sources MoonEP, the
+// Library Used to Train the MoE Model Kimi K3"):
+//   * "Why expert parallelism is needed": maxvio = max_e(T_e / T-bar) - 1;
+//   * "How MoonEP works": every rank gets exactly S*K slots, redundant experts
+//     scheduled online from the current router output;
+//   * "Why this matters to engineers": tokens written straight into
+//     positions grouped by expert, static shapes, no host synchronisation.
+// The schedule is the stable sort of (token, k) pairs by (expert, g, k) cut
+// into R chunks of S*K.
+//
+// Structure.  The pairs are split into `nb` contiguous tiles, one per block
+// (nb <= number of SMs, all co-resident), and each tile into 32 contiguous
+// warp ranges.
+//   Phase 1  every warp builds a private histogram of its range in shared
+//            memory (match_any groups equal expert ids, one leader adds the
+//            group size: no atomics); the block turns the 32 warp histograms
+//            into per-warp exclusive offsets and publishes its tile total per
+//            expert to tile[e][b].
+//   -- grid barrier --
+//   Phase 2  one warp per expert scans its row tile[e][0..nb) into exclusive
+//            per-tile offsets and writes T_e.
+//   -- grid barrier --
+//   Phase 3  every block scans T_e over experts (expert offsets), block 0
+//            writes maxvio, the offsets, segments, CSR pointers and replica
+//            list; every warp walks its range again in (g, k) order and gives
+//            each pair slot = off_e + tile offset + warp offset + rank among
+//            equal ids earlier in the warp (match_any + popc).
+// All the idx reads of phase 3 hit L2 (the plan input is at most a few MB).
+#include <climits>
+#include <cstdint>
+
+#include "mep_device.cuh"
+#include "mep_internal.h"
+
+namespace mep {
+
+namespace {
+
+constexpr int kThreads = kPlanThreads;
+constexpr int kWarps = kThreads / 32;
+constexpr int kBatch = 8;  // coalesced 32-pair loads in flight per warp
+
+struct PlanParams {
+  const int32_t *idx;
+  int32_t R, S, E, K;
+  int64_t NK, SK;
+  int32_t nb;
+  int64_t ppb;  // pairs per tile
+  int32_t full;  // 0: counts + maxvio only
+  int32_t *counts, *expert_offset, *slot, *src_pair;
+  int4 *seg;
+  int32_t *rank_seg_ptr, *expert_seg_ptr, *replica_seg;
+  int32_t *num_seg, *num_replicas, *max_count, *status;
+  double *maxvio;
+  int32_t *tile;   // workspace [E][nb]
+  uint32_t *bar;   // workspace barrier words
+  uint64_t wait_ns;
+};
+
+// Exclusive prefix sum of one value per thread over the block; *total gets the
+// block sum.  Uses s_w[32]; every thread of the block must call it.
+__device__ __forceinline__ int block_excl_scan(int v, int *total, int *s_w) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) s_w[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = s_w[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    s_w[lane] = w;
+  }
+  __syncthreads();
+  const int before = warp ? s_w[warp - 1] : 0;
+  *total = s_w[kWarps - 1];
+  __syncthreads();
+  return before + x - v;
+}
+
+__device__ __forceinline__ int block_max(int v, int *s_w) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
+  if (lane == 0) s_w[warp] = v;
+  __syncthreads();
+  int m = s_w[0];
+  for (int w = 1; w < kWarps; ++w) m = max(m, s_w[w]);
+  __syncthreads();
+  return m;
+}
+
+__global__ void __launch_bounds__(kThreads, 1) plan_kernel(PlanParams p) {
+  extern __shared__ int wh_all[];  // [kWarps][E] per-warp histograms / cursors
+  __shared__ int s_w[32];
+  __shared__ int s_off[MEP_MAX_EXPERTS + 1];
+  __shared__ int s_sbase[MEP_MAX_EXPERTS + 1];
+
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int E = p.E;
+  if (blockIdx.x == 0 && t == 0) *p.status = 0;
+
+  int *wh = wh_all + warp * E;
+  for (int i = t; i < kWarps * E; i += kThreads) wh_all[i] = 0;
+  __syncthreads();
+
+  // Tile and warp ranges.
+  const int64_t b0 = (int64_t)blockIdx.x * p.ppb;
+  const int64_t b1 = min(b0 + p.ppb, p.NK);
+  const int64_t n = b1 > b0 ? b1 - b0 : 0;
+  const int64_t w0 = b0 + (n * warp) / kWarps;
+  const int64_t w1 = b0 + (n * (warp + 1)) / kWarps;
+
+  // ---- phase 1: warp-private histograms ------------------------------------
+  bool bad = false;
+  for (int64_t c = w0; c < w1; c += 32 * kBatch) {
+    int ev[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int64_t q = c + u * 32 + lane;
+      ev[u] = q < w1 ? __ldg(p.idx + q) : INT_MIN;
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      if (c + u * 32 >= w1) break;  // warp-uniform
+      const int64_t q = c + u * 32 + lane;
+      const bool act = q < w1;
+      const int e = ev[u];
+      const bool valid = act && (unsigned)e < (unsigned)E;
+      bad |= act && !valid;
+      const unsigned peers = __match_any_sync(0xffffffffu, valid ? e : -1);
+      if (valid && lane == __ffs(peers) - 1) wh[e] += __popc(peers);
+      __syncwarp();
+    }
+  }
+  __syncthreads();
+  if (t < E) {  // per-warp exclusive offsets inside the tile; tile total
+    int run = 0;
+    for (int w = 0; w < kWarps; ++w) {
+      const int v = wh_all[w * E + t];
+      wh_all[w * E + t] = run;
+      run += v;
+    }
+    __stcg(p.tile + (int64_t)t * p.nb + blockIdx.x, run);
+  }
+  bad = __syncthreads_or(bad);
+
+  if (!grid_barrier(p.bar, p.nb, p.wait_ns, p.status)) return;
+  if (bad && t == 0) set_status(p.status, MEP_ERR_DEVICE_DATA);
+
+  // ---- phase 2: per-expert scan over tiles ----------------------------------
+  {
+    const int per = (p.nb + 31) / 32;
+    for (int e = blockIdx.x * kWarps + warp; e < E; e += p.nb * kWarps) {
+      int32_t *row = p.tile + (int64_t)e * p.nb;
+      const int lo = min(lane * per, p.nb), hi = min(lo + per, p.nb);
+      int s = 0;
+      for (int b = lo; b < hi; ++b) s += __ldcg(row + b);
+      int incl = s;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (p.full) {
+        int run = incl - s;
+        for (int b = lo; b < hi; ++b) {
+          const int v = __ldcg(row + b);
+          __stcg(row + b, run);
+          run += v;
+        }
+      }
+      const int total = __shfl_sync(0xffffffffu, incl, 31);
+      if (lane == 0) __stcg(p.counts + e, total);
+    }
+  }
+
+  if (!grid_barrier(p.bar, p.nb, p.wait_ns, p.status)) return;
+
+  // ---- phase 3: offsets, scalars, segments, scatter -------------------------
+  const int T = t < E ? __ldcg(p.counts + t) : 0;
+  int total;
+  const int off = block_excl_scan(T, &total, s_w);
+
+  if (blockIdx.x == 0) {
+    const int mx = block_max(T, s_w);
+    if (t == 0) {
+      *p.max_count = mx;
+      *p.maxvio = (double)((long long)mx * E) / (double)p.NK - 1.0;
+    }
+  }
+  if (!p.full) return;
+
+  if (blockIdx.x == 0) {
+    const int64_t SK = p.SK;
+    int nseg_e = 0, r0 = 0, r1 = -1;
+    if (t < E && T > 0) {
+      r0 = (int)(off / SK);
+      r1 = (int)((off + (int64_t)T - 1) / SK);
+      nseg_e = r1 - r0 + 1;
+    }
+    int nseg;
+    const int sbase = block_excl_scan(nseg_e, &nseg, s_w);
+    const int home = t / (E / p.R);
+    const int nrep_e = nseg_e - ((nseg_e > 0 && home >= r0 && home <= r1) ? 1 : 0);
+    int nrep;
+    int rbase = block_excl_scan(nrep_e, &nrep, s_w);
+    if (t < E) {
+      s_off[t] = off;
+      s_sbase[t] = sbase;
+      p.expert_offset[t] = off;
+      p.expert_seg_ptr[t] = sbase;
+      for (int j = 0; j < nseg_e; ++j) {
+        const int r = r0 + j;
+        const int64_t lo = max((int64_t)off, (int64_t)r * SK);
+        const int64_t hi = min((int64_t)off + T, (int64_t)(r + 1) * SK);
+        p.seg[sbase + j] = make_int4(t, r, (int)(lo - (int64_t)r * SK), (int)(hi - lo));
+        if (r != home) p.replica_seg[rbase++] = sbase + j;
+      }
+    }
+    if (t == 0) {
+      s_off[E] = total;
+      s_sbase[E] = nseg;
+      p.expert_offset[E] = total;
+      p.expert_seg_ptr[E] = nseg;
+      *p.num_seg = nseg;
+      *p.num_replicas = nrep;
+    }
+    __syncthreads();
+    for (int r = t; r <= p.R; r += kThreads) {
+      const int64_t x = (int64_t)r * SK;
+      int ptr = nseg;
+      if (r < p.R && x < total) {
+        int lo = 0, hi = E + 1;  // first index with s_off > x
+        while (lo < hi) {
+          const int mid = (lo + hi) >> 1;
+          if ((int64_t)s_off[mid] <= x) lo = mid + 1; else hi = mid;
+        }
+        const int e = lo - 1;
+        ptr = s_sbase[e] + (r - (int)(s_off[e] / SK));
+      }
+      p.rank_seg_ptr[r] = ptr;
+    }
+  }
+
+  // Per-warp cursors: expert offset + tile offset + warp offset.
+  if (t < E) {
+    const int base = off + __ldcg(p.tile + (int64_t)t * p.nb + blockIdx.x);
+    for (int w = 0; w < kWarps; ++w) wh_all[w * E + t] += base;
+  }
+  __syncthreads();
+
+  const unsigned lt = lanemask_lt();
+  for (int64_t c = w0; c < w1; c += 32 * kBatch) {
+    int ev[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int64_t q = c + u * 32 + lane;
+      ev[u] = q < w1 ? __ldg(p.idx + q) : INT_MIN;
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      if (c + u * 32 >= w1) break;
+      const int64_t q = c + u * 32 + lane;
+      const bool act = q < w1;
+      const int e = ev[u];
+      const bool valid = act && (unsigned)e < (unsigned)E;
+      const unsigned peers = __match_any_sync(0xffffffffu, valid ? e : -1);
+      const int base = valid ? wh[e] : 0;
+      __syncwarp();
+      if (valid) {
+        const int s = base + __popc(peers & lt);
+        p.slot[q] = s;
+        if ((unsigned)s < (unsigned)p.NK) p.src_pair[s] = (int32_t)q;
+        if (lane == __ffs(peers) - 1) wh[e] = base + __popc(peers);
+      } else if (act) {
+        p.slot[q] = -1;
+      }
+      __syncwarp();
+    }
+  }
+}
+
+struct PlanDev {
+  int sms = 0;
+  int max_blocks = 0;  // co-resident plan blocks (cooperative grid limit)
+  int smem_attr = -1;  // dynamic smem size the attribute was set for
+};
+
+PlanDev g_plan_dev[64];
+
+}  // namespace
+
+size_t plan_workspace_bytes(const mep_shape_t &s) {
+  return kPlanWsHeader + (size_t)s.E * kPlanMaxBlocks * sizeof(int32_t);
+}
+
+cudaError_t launch_plan(const mep_shape_t &s, const int32_t *idx, const mep_plan_t &pl,
+                        int full, void *ws, uint64_t wait_ns, cudaStream_t stream) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  PlanDev &d = g_plan_dev[dev];
+  const size_t smem = (size_t)kWarps * s.E * sizeof(int);
+  if (d.smem_attr != (int)smem) {
+    err = cudaFuncSetAttribute(plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    err = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+    if (err != cudaSuccess) return err;
+    int per_sm = 0;
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, plan_kernel, kThreads, smem);
+    if (err != cudaSuccess) return err;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    d.max_blocks = per_sm * d.sms;
+    d.smem_attr = (int)smem;
+  }
+  const int64_t NK = (int64_t)s.R * s.S * s.K;
+  int64_t want = (NK + kPlanMinPairsPerBlock - 1) / kPlanMinPairsPerBlock;
+  int nb = (int)std::min<int64_t>(std::max<int64_t>(want, 1),
+                                  std::min(d.max_blocks, kPlanMaxBlocks));
+  PlanParams p{};
+  p.idx = idx;
+  p.R = s.R; p.S = s.S; p.E = s.E; p.K = s.K;
+  p.NK = NK;
+  p.SK = (int64_t)s.S * s.K;
+  p.nb = nb;
+  p.ppb = (NK + nb - 1) / nb;
+  p.full = full;
+  p.counts = pl.counts; p.expert_offset = pl.expert_offset; p.slot = pl.slot;
+  p.src_pair = pl.src_pair; p.seg = reinterpret_cast<int4 *>(pl.seg);
+  p.rank_seg_ptr = pl.rank_seg_ptr; p.expert_seg_ptr = pl.expert_seg_ptr;
+  p.replica_seg = pl.replica_seg; p.num_seg = pl.num_seg; p.num_replicas = pl.num_replicas;
+  p.max_count = pl.max_count; p.status = pl.status; p.maxvio = pl.maxvio;
+  p.bar = reinterpret_cast<uint32_t *>(ws);
+  p.tile = reinterpret_cast<int32_t *>(static_cast<char *>(ws) + kPlanWsHeader);
+  p.wait_ns = wait_ns;
+
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(nb);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, plan_kernel, p);
+}
+
+}  // namespace mep
