@@ -53,6 +53,10 @@ def parse_args():
     ap.add_argument("--impl", choices=["mep", "reference"], default="mep")
     ap.add_argument("--workload", default=workloads.BENCH_WORKLOAD,
                     choices=list(workloads.WORKLOADS))
+    ap.add_argument("--S", type=int, default=None,
+                    help="tokens per rank (default: the workload's); for small profiling cases")
+    ap.add_argument("--P", type=int, default=None,
+                    help="gradient row length (default: the workload's); for small profiling cases")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
@@ -247,6 +251,8 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
     wl = workloads.WORKLOADS[args.workload]
+    if args.S is not None or args.P is not None:
+        wl = workloads.reduced(wl, S=args.S or wl.S, P=args.P if args.P is not None else wl.P)
     R, S, E, K, H, P, N, NK = wl.R, wl.S, wl.E, wl.K, wl.H, wl.P, wl.N, wl.NK
     s = mep.Shape(R, S, E, K)
     idx_h, w_h = workloads.routing(wl, seed=0)
