@@ -6,16 +6,16 @@
  *
  *   "Moonshot AI Open-Sources MoonEP, the Library Used to Train the MoE Model
  *   Kimi K3" (below: the MoonEP release page)
- *     - "Why expert parallelism is needed": the router sends every token to
- *       its top-K experts; skew is measured as maxvio = max_e(T_e / T-bar) - 1,
- *       zero being perfect balance.
- *     - "How MoonEP works": every EP rank receives exactly S x K tokens however
- *       skewed the routing; a small number of redundant experts are scheduled
- *       online from the current router output; their gradients are reduced
- *       back to the home ranks on the backward pass.
- *     - "Why this matters to engineers": static buffer shapes and zero-copy --
- *       tokens are written straight into positions grouped by expert, with no
- *       per-layer host synchronisation.
+ *     - "Why expert parallelism is needed": a router assigns each token to K
+ *       experts; imbalance is measured by maxvio = max_e(T_e / T-bar) - 1,
+ *       which is 0 for a perfectly even load.
+ *     - "How MoonEP works": the number of token slots per EP rank is pinned
+ *       at S x K whatever the routing; a few duplicate (replica) experts are
+ *       placed each step from that step's routing, and in the backward pass
+ *       the duplicates' gradients are summed into the home copy.
+ *     - "Why this matters to engineers": fixed buffer shapes, no staging
+ *       copy -- each row goes directly to its final expert-ordered slot --
+ *       and no host round trip per layer.
  *   "Moonshot AI Open-Sources MoonEP: A Perfectly Balanced Expert Parallelism
  *   Library for MoE Training", "The problem MoonEP targets": T_e counts the
  *   tokens routed to expert e; T-bar is the count expected under perfect
@@ -140,13 +140,13 @@ MEP_API mep_status_t mep_maxvio(mep_shape_t shape, const int32_t *topk_idx,
  *             (g, k) order with the same expert e}; src_pair its inverse;
  *             the segments, CSR pointers and replica list of the R-way cut.
  *             plan->status is cleared at the start of the call.
- * Each rank r receives exactly SK slots, [r*SK, (r+1)*SK), grouped by expert. */
+ * Rank r holds exactly the SK slots [r*SK, (r+1)*SK), in expert order. */
 MEP_API mep_status_t mep_plan(mep_shape_t shape, const int32_t *topk_idx,
                       const mep_plan_t *plan, void *ws, size_t ws_bytes,
                       void *stream);
 
 /* Zero-copy dispatch into the static receive buffer ("Why this matters to
- * engineers": tokens written straight into positions grouped by expert).
+ * engineers": each row is copied directly to its final expert-ordered slot).
  *   x    bf16 [N, H], 16-byte aligned; H % 8 == 0, 8 <= H <= MEP_MAX_HIDDEN.
  *   buf  bf16 [R, S*K, H] out, 16-byte aligned: buf[slot[g,k], :] = x[g, :]
  *        for every pair; a token routed to several experts is copied once
@@ -166,7 +166,7 @@ MEP_API mep_status_t mep_combine(mep_shape_t shape, int32_t H, const mep_plan_t 
                          void *stream);
 
 /* Backward reduction of replica weight-gradients into their home expert
- * ("How MoonEP works": gradients reduced back to the home ranks).
+ * ("How MoonEP works": duplicates' gradients summed into the home copy).
  *   seg_grads  float32 [E+R-1, P]: row s is the gradient computed by segment
  *              s of the plan (its rank's copy of expert seg[s].expert); rows
  *              s >= num_seg are ignored.  16-byte aligned when P % 4 == 0.

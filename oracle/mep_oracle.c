@@ -12,19 +12,19 @@
  * Sources, by page title and section:
  *   [P1-why]  "Moonshot AI Open-Sources MoonEP, the Library Used to Train the
  *             MoE Model Kimi K3", section "Why expert parallelism is needed":
- *             the router sends each token to its top-K experts; skew metric
- *             maxvio = max_e(T_e / T-bar) - 1, zero meaning perfect balance.
+ *             a router assigns each token to K experts; the imbalance metric
+ *             maxvio = max_e(T_e / T-bar) - 1 is 0 for an even load.
  *   [P2-prob] "Moonshot AI Open-Sources MoonEP: A Perfectly Balanced Expert
  *             Parallelism Library for MoE Training", section "The problem
  *             MoonEP targets": T_e is the number of tokens routed to expert e,
  *             T-bar the count expected under perfect balance.
- *   [P1-how]  first title, section "How MoonEP works": every rank receives
- *             exactly S x K tokens; a few redundant experts are scheduled
- *             online from the current router output; their gradients are
- *             reduced back to the home ranks on the backward pass.
- *   [P1-eng]  first title, section "Why this matters to engineers": static
- *             buffer shapes, zero-copy, tokens written straight into
- *             positions grouped by expert; section "Key facts": B = E/R for
+ *   [P1-how]  first title, section "How MoonEP works": a rank's share is
+ *             pinned at S x K token slots; a few duplicate experts are placed
+ *             per step from that step's routing; in the backward pass their
+ *             gradients are summed into the home copy.
+ *   [P1-eng]  first title, section "Why this matters to engineers": fixed
+ *             buffer shapes, no staging copy, each row lands directly in its
+ *             expert-ordered slot; section "Key facts": B = E/R for
  *             training.
  *
  * Readings where the pages are silent (each is also listed in the design

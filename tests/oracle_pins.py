@@ -10,7 +10,7 @@ a mismatch.  The pins rest on
   * closed forms (round-robin routing gives maxvio = 0 and no replicas;
     adversarial routing gives maxvio = 31 and 31 replicas at the skew shape);
   * invariants the pages fix (exactly S*K slots per rank, every (token,k)
-    placed once, slots grouped by expert, counts sum to R*S*K);
+    placed once, slots in expert order, counts sum to R*S*K);
   * a library routine (torch's float32 -> bf16 conversion).
 They are kept in one module so ``test_oracle_mutants.py`` can rerun the whole
 set against oracles with planted mistakes.
@@ -226,7 +226,7 @@ def check_plan_invariants(pl, R, S, E, K, idx):
     # every (token, k) placed exactly once: slot is a bijection, src its inverse
     assert np.array_equal(np.sort(slot), np.arange(NK))
     assert np.array_equal(src[slot], np.arange(NK))
-    # grouped by expert, in (g, k) order inside an expert (stability)
+    # expert order, and (g, k) order inside an expert (stability)
     e_of_p = idx[src]
     assert np.all(np.diff(e_of_p) >= 0)
     same = np.diff(e_of_p) == 0

@@ -2,9 +2,9 @@
 //   out[g, :] = bf16_rne( sum_{k=0..K-1} w[g,k] * y[slot[g,k], :] )
 // accumulated in float32 with one fused multiply-add per term, k ascending.
 //
-// Method: the router sends each token to its top-K experts (MoonEP release
-// page, "Why expert parallelism is needed"); the expert outputs come back to
-// the token's position weighted by the router weights.
+// Method: a router assigns every token to K experts (MoonEP release page,
+// "Why expert parallelism is needed"); the K expert outputs return to the
+// token's position, weighted by the router weights.
 //
 // Each thread owns one 16-byte column chunk (8 bf16) of one token: it loads
 // the token's K slot ids and weights (shared by the warp, served by L1), then

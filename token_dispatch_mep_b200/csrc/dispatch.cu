@@ -1,8 +1,9 @@
 // Zero-copy dispatch: buf[slot[g,k], :] = x[g, :] for every (token, k) pair.
 //
-// Method: tokens are written straight into positions grouped by expert, into
-// a receive buffer whose shape never changes (MoonEP release page, "Why this
-// matters to engineers"; "How MoonEP works": exactly S*K slots per rank).
+// Method: each token row is copied once per routed expert, directly into its
+// final slot of an expert-ordered receive buffer whose shape never changes
+// (MoonEP release page, "Why this matters to engineers"; "How MoonEP works":
+// a fixed S*K slots per rank).
 //
 // Token-major, so each hidden row crosses HBM once on the way in and K times
 // on the way out (the algorithmic minimum).  Each warp runs its own pipeline

@@ -3,11 +3,12 @@
 //
 // The method (MoonEP release page "Moonshot AI Open-Sources MoonEP, the
 // Library Used to Train the MoE Model Kimi K3"):
-//   * "Why expert parallelism is needed": maxvio = max_e(T_e / T-bar) - 1;
-//   * "How MoonEP works": every rank gets exactly S*K slots, redundant experts
-//     scheduled online from the current router output;
-//   * "Why this matters to engineers": tokens written straight into
-//     positions grouped by expert, static shapes, no host synchronisation.
+//   * "Why expert parallelism is needed": the skew metric
+//     maxvio = max_e(T_e / T-bar) - 1;
+//   * "How MoonEP works": each rank's share is fixed at S*K slots, and a few
+//     duplicate experts are placed per step from that step's routing;
+//   * "Why this matters to engineers": each row goes directly to its final,
+//     expert-ordered slot in a buffer of fixed shape, without a host round trip.
 // The schedule is the stable sort of (token, k) pairs by (expert, g, k) cut
 // into R chunks of S*K.
 //

@@ -2,10 +2,11 @@
 //   home[e, :] = sum over expert e's segments s (ascending) of G[s, :]
 // in float32, zero for an expert with no segment.
 //
-// Method: "on the backward pass their gradients are reduced back to the
-// 'home' ranks" (MoonEP release page, "How MoonEP works").  The plan lists an
-// expert's segments contiguously (expert_seg_ptr), so the reduction is a
-// segmented sum over contiguous rows of G.
+// Method: during the backward pass the gradients of an expert's duplicates are
+// summed into the copy on its home rank (MoonEP release page, "How MoonEP
+// works").  The plan lists an expert's segments contiguously
+// (expert_seg_ptr), so the reduction is a segmented sum over contiguous rows
+// of G.
 //
 // Flat grid-stride over (expert, column) items, expert-major, so consecutive
 // threads read consecutive 16-byte columns.  Each thread issues up to eight
