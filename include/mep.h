@@ -178,6 +178,26 @@ MEP_API mep_status_t mep_reduce_replica_grads(mep_shape_t shape, const mep_plan_
                                       int64_t P, const float *seg_grads,
                                       float *home_grads, void *stream);
 
+/* mep_plan without a caller-supplied workspace, for callers that cannot
+ * allocate device memory (no allocator in their runtime, or a host framework
+ * that owns the device memory pool and forbids allocation after start-up).
+ * The paper (the MoonEP release pages) has no counterpart to this call.
+ * Same arguments and results as mep_plan.  Its scratch is a device array of
+ * MEP_NOALLOC_SCRATCH_BYTES compiled into the library, held by every GPU that
+ * loads the library until the process exits.  It holds the workspace of
+ * the largest shape the library accepts (E = MEP_MAX_EXPERTS); a shape beyond
+ * the shape rules is rejected with MEP_ERR_INVALID_ARG, and a workspace that
+ * would not fit the array with MEP_ERR_WORKSPACE, before anything runs.  The first
+ * call on a device looks up that array's device address (make that call
+ * before any stream capture on the device).  Each call clears the array's
+ * barrier words with a 256-byte memset on `stream`, then launches the plan.
+ * The array is shared by all calls on a device: calls that overlap on the GPU
+ * (e.g. on two streams with no ordering between them) race and give
+ * undefined plans.  Allocates nothing and frees nothing. */
+#define MEP_NOALLOC_SCRATCH_BYTES (256u + 1024u * 1024u * 4u)
+MEP_API mep_status_t mep_plan_noalloc(mep_shape_t shape, const int32_t *topk_idx,
+                                      const mep_plan_t *plan, void *stream);
+
 /* Synchronises `stream` and returns the plan's device status word (MEP_OK if
  * every call so far on this plan ran clean), or MEP_ERR_CUDA if the copy
  * itself fails.  The only call that blocks the host. */

@@ -18,7 +18,8 @@ import torch
 
 __all__ = [
     "MepError", "Shape", "Plan", "load_library", "library_path",
-    "mep_plan_workspace_bytes", "mep_maxvio", "mep_plan", "mep_dispatch", "mep_combine",
+    "mep_plan_workspace_bytes", "mep_maxvio", "mep_plan", "mep_plan_noalloc", "mep_dispatch",
+    "mep_combine",
     "mep_reduce_replica_grads", "mep_read_status", "mep_status_string",
     "mep_set_wait_limit_ns", "mep_get_wait_limit_ns", "mep_version", "STATUS",
 ]
@@ -32,7 +33,8 @@ STATUS = {0: "MEP_OK", 1: "MEP_ERR_INVALID_ARG", 2: "MEP_ERR_MISALIGNED", 3: "ME
 # Symbols the header declares; the CPU test suite checks they are exported.
 ABI_SYMBOLS = ("mep_plan_workspace_bytes", "mep_maxvio", "mep_plan", "mep_dispatch", "mep_combine",
                "mep_reduce_replica_grads", "mep_read_status", "mep_status_string",
-               "mep_set_wait_limit_ns", "mep_get_wait_limit_ns", "mep_version")
+               "mep_set_wait_limit_ns", "mep_get_wait_limit_ns", "mep_version",
+               "mep_plan_noalloc")
 
 
 class MepError(RuntimeError):
@@ -103,6 +105,7 @@ def load_library():
         "mep_set_wait_limit_ns": ([u64], None),
         "mep_get_wait_limit_ns": ([], u64),
         "mep_version": ([], i32),
+        "mep_plan_noalloc": ([Shape, vp, P, vp], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -220,6 +223,17 @@ def mep_plan(shape, topk_idx, plan: Plan, workspace=None):
     ws_t = plan.workspace if workspace is None else workspace
     ws = _need(ws_t, "workspace", torch.uint8, mep_plan_workspace_bytes(s), dev)
     _ok(L.mep_plan(s, idx, ctypes.byref(plan.struct), ws, ws_t.numel(), _stream(dev)), "mep_plan")
+
+
+def mep_plan_noalloc(shape, topk_idx, plan: Plan):
+    """``mep_plan`` without a workspace argument: for callers that cannot
+    allocate device memory.  The library's own static device scratch is used
+    instead (shared by every call on the device; calls that overlap on the
+    GPU race)."""
+    L, s = load_library(), _shape(shape)
+    dev = plan.device
+    idx = _need(topk_idx, "topk_idx", torch.int32, s.NK, dev)
+    _ok(L.mep_plan_noalloc(s, idx, ctypes.byref(plan.struct), _stream(dev)), "mep_plan_noalloc")
 
 
 def mep_dispatch(shape, H: int, plan: Plan, x, buf):
