@@ -155,6 +155,25 @@ class ClockSampler:
                 "samples": len(self.samples)}
 
 
+# ------------------------------------------------------------- multi-rank
+
+def max_over_ranks(value: float, world: int, device) -> float:
+    """Max of a per-rank float over all ranks (the step time of the slowest
+    replica); a no-op for one rank."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(tokens_per_rank: int, world: int, ms: float) -> float:
+    """Tokens per second of all replicas together, timed by the slowest."""
+    return tokens_per_rank * world / (ms * 1e-3)
+
+
 # ------------------------------------------------------------ CPU oracle leg
 
 def oracle_throughput(wl, target_seconds: float, host=None):
@@ -311,12 +330,8 @@ def main():
 
     stage = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)]
                       for i in range(args.steps)])          # ms
-    ms_step = float(stage.sum(axis=1).mean())
-    if world > 1:
-        t = torch.tensor([ms_step], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step = float(t.item())
-    value = N * world / (ms_step * 1e-3)
+    ms_step = max_over_ranks(float(stage.sum(axis=1).mean()), world, dev)
+    value = whole_job_rate(N, world, ms_step)
 
     stage_ms = dict(zip(["plan", "dispatch", "combine", "reduce"], stage.mean(axis=0).tolist()))
     algo = {
@@ -378,14 +393,10 @@ def main():
             e2e_step()
         e1.record()
         torch.cuda.synchronize()
-        ms_e2e = e0.elapsed_time(e1) / args.e2e_steps
-        if world > 1:
-            t = torch.tensor([ms_e2e], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms_e2e = float(t.item())
+        ms_e2e = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, world, dev)
         if int(hsc[3].item()) != 0:
             raise RuntimeError("device status not OK after e2e steps")
-        e2e = {"value": N * world / (ms_e2e * 1e-3), "unit": "tokens/s",
+        e2e = {"value": whole_job_rate(N, world, ms_e2e), "unit": "tokens/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e}
 
     cpu = None
@@ -413,7 +424,7 @@ def main():
             "stages_ms": stage_ms,
             "kernels": kernels,
             "plan_us": stage_ms["plan"] * 1e3,
-            "pdc_tokens_per_s": N * world / (pdc_ms * 1e-3),
+            "pdc_tokens_per_s": whole_job_rate(N, world, pdc_ms),
             "num_seg": num_seg,
         }
         print(json.dumps(line), flush=True)
