@@ -29,8 +29,8 @@ def _stale(out: str, deps) -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def _compile(src: str, extra) -> str:
-    obj = os.path.join(OBJDIR, os.path.splitext(src)[0] + ".o")
+def _compile(src: str, extra, objdir: str = OBJDIR) -> str:
+    obj = os.path.join(objdir, os.path.splitext(src)[0] + ".o")
     deps = [os.path.join(CSRC, src), os.path.join(INCLUDE, "mep.h")] + \
         [os.path.join(CSRC, h) for h in HEADERS]
     if _stale(obj, deps):
@@ -38,21 +38,24 @@ def _compile(src: str, extra) -> str:
     return obj
 
 
-def build(verbose_ptxas: bool = False, force: bool = False) -> str:
-    """Compile every kernel source for sm_100a and link ``libmep.so`` next to
-    this file.  Returns the library path."""
-    os.makedirs(OBJDIR, exist_ok=True)
+def build(verbose_ptxas: bool = False, force: bool = False, defines=(), lib: str = LIB,
+          objdir: str = OBJDIR) -> str:
+    """Compile every kernel source for sm_100a and link ``libmep.so`` (next to
+    this file unless `lib` says otherwise).  `defines` are extra -D tunables
+    (launch shapes); the default build uses none.  Returns the library path."""
+    os.makedirs(objdir, exist_ok=True)
     extra = ["-Xptxas", "-v"] if verbose_ptxas else []
+    extra += [f"-D{d}" for d in defines]
     if force:
-        for f in os.listdir(OBJDIR):
+        for f in os.listdir(objdir):
             if f.endswith(".o"):
-                os.remove(os.path.join(OBJDIR, f))
+                os.remove(os.path.join(objdir, f))
     with concurrent.futures.ThreadPoolExecutor(len(SOURCES)) as ex:
-        objs = list(ex.map(lambda s: _compile(s, extra), SOURCES))
-    if force or _stale(LIB, objs):
+        objs = list(ex.map(lambda s: _compile(s, extra, objdir), SOURCES))
+    if force or _stale(lib, objs):
         subprocess.run([NVCC, "-shared", "-gencode", "arch=compute_100a,code=sm_100a",
-                        "-o", LIB, *objs], check=True)
-    return LIB
+                        "-o", lib, *objs], check=True)
+    return lib
 
 
 if __name__ == "__main__":

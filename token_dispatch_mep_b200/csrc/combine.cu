@@ -6,11 +6,14 @@
 // "Why expert parallelism is needed"); the K expert outputs return to the
 // token's position, weighted by the router weights.
 //
-// Each thread owns one 16-byte column chunk (8 bf16) of one token: it loads
-// the token's K slot ids and weights (shared by the warp, served by L1), then
-// issues the K independent 16-byte row loads before it touches any of them,
-// so K x 16 bytes per thread are in flight.  Expert outputs are read once
-// (streaming loads); the output row is written once (streaming stores).
+// Work unit: a warp task = one token and a run of 32 x kU 16-byte column
+// chunks of its row (lane l owns chunks l, l+32, ...).  Lanes k < K load the
+// token's slot id and weight once and the warp broadcasts them with
+// shuffles; the next task's slot ids and weights are fetched before the
+// current task's rows, so the two dependent loads of consecutive tasks
+// overlap.  Each lane then issues all K x kU independent 16-byte streaming
+// loads before it touches any of them, adds them in k order with float32
+// FMAs, rounds to bf16 and writes 16 bytes per chunk (streaming store).
 #include <algorithm>
 #include <cstdint>
 
@@ -19,11 +22,25 @@
 #include "mep_device.cuh"
 #include "mep_internal.h"
 
+#ifndef MEP_COMBINE_LOADS
+#define MEP_COMBINE_LOADS 16  // 16-byte row loads in flight per lane (K x kU)
+#endif
+#ifndef MEP_COMBINE_MAX_U
+#define MEP_COMBINE_MAX_U 2  // 16-byte chunks per lane per task, at most
+#endif
+#ifndef MEP_COMBINE_BLOCKS_PER_SM
+#define MEP_COMBINE_BLOCKS_PER_SM 4
+#endif
+#ifndef MEP_COMBINE_MIN_BLOCKS
+#define MEP_COMBINE_MIN_BLOCKS 2  // launch bound: resident blocks per SM
+#endif
+
 namespace mep {
 
 namespace {
 
 constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
 
 struct CombineParams {
   const uint16_t *y;
@@ -31,10 +48,10 @@ struct CombineParams {
   const int32_t *slot;
   uint16_t *out;
   int32_t *status;
-  int64_t NK;
+  int64_t N, NK;
   int32_t K, H;
-  uint32_t chunks_per_row;  // H / 8
-  uint64_t items;           // N * H / 8
+  int32_t chunks;      // 16-byte chunks per row = H / 8
+  int32_t parts;       // warp tasks per token
 };
 
 __device__ __forceinline__ void fma8(float (&acc)[8], float wk, const uint4 &v) {
@@ -58,46 +75,82 @@ __device__ __forceinline__ uint4 pack8(const float (&acc)[8]) {
   return make_uint4(u[0], u[1], u[2], u[3]);
 }
 
-template <int KC>
-__global__ void __launch_bounds__(kThreads) combine_kernel(CombineParams p) {
-  const uint64_t stride = (uint64_t)gridDim.x * kThreads;
+template <int KC, int U>
+__global__ void __launch_bounds__(kThreads, MEP_COMBINE_MIN_BLOCKS) combine_kernel(CombineParams p) {
+  const int lane = threadIdx.x & 31;
+  const int64_t nwarps = (int64_t)gridDim.x * kWarps;
+  const int64_t ntask = p.N * p.parts;
+  int64_t task = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
   bool bad = false;
-  for (uint64_t it = (uint64_t)blockIdx.x * kThreads + threadIdx.x; it < p.items; it += stride) {
-    const uint64_t g = it / p.chunks_per_row;
-    const uint32_t c = (uint32_t)(it - g * p.chunks_per_row);
-    int pk[KC];
-    float wk[KC];
-#pragma unroll
-    for (int k = 0; k < KC; ++k) {
-      if (k < p.K) {
-        pk[k] = __ldg(p.slot + g * p.K + k);
-        wk[k] = __ldg(p.w + g * p.K + k);
-      }
+
+  // slot id and weight of (token of `task`, k = lane) for lanes < K
+  auto fetch = [&](int64_t t, int &sl, float &wt) {
+    sl = -1;
+    wt = 0.f;
+    if (t < ntask && lane < p.K) {
+      const int64_t g = t / p.parts;
+      sl = __ldg(p.slot + g * p.K + lane);
+      wt = __ldg(p.w + g * p.K + lane);
     }
-    uint4 v[KC];
+  };
+  int sl, nsl;
+  float wt, nwt;
+  fetch(task, sl, wt);
+
+  for (; task < ntask; task += nwarps) {
+    fetch(task + nwarps, nsl, nwt);
+    const int64_t g = task / p.parts;
+    const int cbase = (int)(task - g * p.parts) * 32 * U + lane;
+    uint4 v[KC][U];
 #pragma unroll
     for (int k = 0; k < KC; ++k) {
+      const int pk = __shfl_sync(0xffffffffu, sl, k);
       if (k < p.K) {
-        if ((unsigned)pk[k] < (unsigned)p.NK) {
-          v[k] = __ldcs(reinterpret_cast<const uint4 *>(p.y + (int64_t)pk[k] * p.H) + c);
-        } else {
-          v[k] = make_uint4(0, 0, 0, 0);
-          bad = true;
+        const bool ok = (unsigned)pk < (unsigned)p.NK;
+        bad |= !ok;
+        const uint4 *row = reinterpret_cast<const uint4 *>(p.y + (int64_t)(ok ? pk : 0) * p.H);
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int c = cbase + u * 32;
+          v[k][u] = (ok && c < p.chunks) ? __ldcs(row + c) : make_uint4(0, 0, 0, 0);
         }
       }
     }
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    float acc[U][8];
 #pragma unroll
-    for (int k = 0; k < KC; ++k)
-      if (k < p.K) fma8(acc, wk[k], v[k]);
-    __stcs(reinterpret_cast<uint4 *>(p.out + g * p.H) + c, pack8(acc));
+    for (int u = 0; u < U; ++u)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[u][j] = 0.f;
+#pragma unroll
+    for (int k = 0; k < KC; ++k) {
+      const float wk = __shfl_sync(0xffffffffu, wt, k);
+      if (k < p.K) {
+#pragma unroll
+        for (int u = 0; u < U; ++u) fma8(acc[u], wk, v[k][u]);
+      }
+    }
+    uint4 *orow = reinterpret_cast<uint4 *>(p.out + g * p.H);
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int c = cbase + u * 32;
+      if (c < p.chunks) __stcs(orow + c, pack8(acc[u]));
+    }
+    sl = nsl;
+    wt = nwt;
   }
   if (bad) set_status(p.status, MEP_ERR_DEVICE_DATA);
 }
 
 template <int KC>
-cudaError_t launch_kc(const CombineParams &p, int blocks, cudaStream_t stream) {
-  combine_kernel<KC><<<blocks, kThreads, 0, stream>>>(p);
+cudaError_t launch_kc(CombineParams p, int sms, cudaStream_t stream) {
+  constexpr int U0 = (MEP_COMBINE_LOADS / KC) > 0 ? (MEP_COMBINE_LOADS / KC) : 1;
+  constexpr int U = U0 < MEP_COMBINE_MAX_U ? U0 : MEP_COMBINE_MAX_U;
+  p.parts = (p.chunks + 32 * U - 1) / (32 * U);
+  const int64_t ntask = p.N * p.parts;
+  const int64_t want = (ntask + kWarps - 1) / kWarps;
+  const int blocks = (int)std::max<int64_t>(
+      1, std::min<int64_t>(want, (int64_t)sms * MEP_COMBINE_BLOCKS_PER_SM));
+  combine_kernel<KC, U><<<blocks, kThreads, 0, stream>>>(p);
   return cudaGetLastError();
 }
 
@@ -117,18 +170,15 @@ cudaError_t launch_combine(const mep_shape_t &s, int32_t H, const mep_plan_t &pl
   p.slot = pl.slot;
   p.out = out;
   p.status = pl.status;
-  const int64_t N = (int64_t)s.R * s.S;
-  p.NK = N * s.K;
+  p.N = (int64_t)s.R * s.S;
+  p.NK = p.N * s.K;
   p.K = s.K;
   p.H = H;
-  p.chunks_per_row = (uint32_t)(H / 8);
-  p.items = (uint64_t)N * p.chunks_per_row;
-  const uint64_t want = (p.items + kThreads - 1) / kThreads;
-  const int blocks = (int)std::max<uint64_t>(1, std::min<uint64_t>(want, (uint64_t)sms * 8));
-  if (s.K <= 2) return launch_kc<2>(p, blocks, stream);
-  if (s.K <= 4) return launch_kc<4>(p, blocks, stream);
-  if (s.K <= 8) return launch_kc<8>(p, blocks, stream);
-  return launch_kc<16>(p, blocks, stream);
+  p.chunks = H / 8;
+  if (s.K <= 2) return launch_kc<2>(p, sms, stream);
+  if (s.K <= 4) return launch_kc<4>(p, sms, stream);
+  if (s.K <= 8) return launch_kc<8>(p, sms, stream);
+  return launch_kc<16>(p, sms, stream);
 }
 
 }  // namespace mep

@@ -25,8 +25,15 @@ namespace mep {
 
 namespace {
 
-constexpr int kMaxWarps = 4;
-constexpr int kMaxStages = 16;
+#ifndef MEP_DISPATCH_WARPS
+#define MEP_DISPATCH_WARPS 4  // independent pipelines (warps) per block
+#endif
+#ifndef MEP_DISPATCH_STAGES
+#define MEP_DISPATCH_STAGES 16  // shared-memory stages per pipeline, at most
+#endif
+
+constexpr int kMaxWarps = MEP_DISPATCH_WARPS;
+constexpr int kMaxStages = MEP_DISPATCH_STAGES;
 constexpr int kMaxK = 16;
 
 struct DispatchParams {
