@@ -207,9 +207,9 @@ MEP_API mep_status_t mep_read_status(const mep_plan_t *plan, void *stream);
 MEP_API const char *mep_status_string(mep_status_t status);
 
 /* Upper bound, in nanoseconds of the GPU global timer, on every device-side
- * wait (grid barriers in the plan, transfer barriers in dispatch).  A wait
- * that runs out records MEP_ERR_TIMEOUT and the kernel returns.  Process-wide;
- * default 1e9 (one second); values below 1000 are raised to 1000. */
+ * wait (the grid barriers of mep_plan and mep_maxvio).  A wait that runs out
+ * records MEP_ERR_TIMEOUT and the kernel returns.  Process-wide; default 1e9
+ * (one second); values below 1000 are raised to 1000. */
 MEP_API void mep_set_wait_limit_ns(uint64_t ns);
 MEP_API uint64_t mep_get_wait_limit_ns(void);
 

@@ -231,16 +231,17 @@ def test_out_of_range_ids_reported_not_fatal(ora):
 
 
 def test_barrier_wait_runs_out_and_recovers(ora):
-    """A grid barrier whose arrival count is poisoned never opens: every block
-    gives up after the wait limit, the status says MEP_ERR_TIMEOUT, and the
-    context stays usable."""
+    """A grid barrier whose arrival count is poisoned (a large negative value,
+    so it can never reach its target) never opens: every block gives up after
+    the wait limit, the status says MEP_ERR_TIMEOUT, and the context stays
+    usable."""
     R, S, E, K = 8, 4096, 64, 6
     idx, _ = _edge_routing(R, S, E, K, "random")
     s = mep.Shape(R, S, E, K)
     plan = mep.Plan(s, DEV)
     old = mep.mep_get_wait_limit_ns()
     try:
-        plan.workspace[:4].view(torch.int32).fill_(1 << 30)
+        plan.workspace[:4].view(torch.int32).fill_(-(1 << 31))
         mep.mep_set_wait_limit_ns(2_000_000)
         mep.mep_plan(s, torch.from_numpy(idx).to(DEV), plan)
         assert mep.mep_read_status(plan) == 6

@@ -94,7 +94,7 @@ mep_status_t mep_dispatch(mep_shape_t shape, int32_t H, const mep_plan_t *plan, 
   if ((st = check_hidden(H)) != MEP_OK) return st;
   if (!plan || !plan->slot || !plan->status || !x || !buf) return MEP_ERR_INVALID_ARG;
   if (!aligned(x, 16) || !aligned(buf, 16) || !aligned(plan->slot, 4)) return MEP_ERR_MISALIGNED;
-  return from_cuda(mep::launch_dispatch(shape, H, *plan, x, buf, g_wait_ns.load(), as_stream(stream)));
+  return from_cuda(mep::launch_dispatch(shape, H, *plan, x, buf, as_stream(stream)));
 }
 
 mep_status_t mep_combine(mep_shape_t shape, int32_t H, const mep_plan_t *plan, const uint16_t *y,

@@ -12,6 +12,7 @@ namespace mep {
 
 constexpr int kPlanThreads = 1024;
 constexpr int kPlanMaxBlocks = 1024;          // bound used to size the workspace
+constexpr int kPlanIdsPerWarp = 512;          // expert ids a plan warp keeps in shared memory
 constexpr int64_t kPlanMinPairsPerBlock = 4096;
 constexpr size_t kPlanWsHeader = 256;         // grid-barrier words
 
@@ -22,8 +23,7 @@ cudaError_t launch_plan(const mep_shape_t &s, const int32_t *idx, const mep_plan
                         int full, void *ws, uint64_t wait_ns, cudaStream_t stream);
 
 cudaError_t launch_dispatch(const mep_shape_t &s, int32_t H, const mep_plan_t &pl,
-                            const uint16_t *x, uint16_t *buf, uint64_t wait_ns,
-                            cudaStream_t stream);
+                            const uint16_t *x, uint16_t *buf, cudaStream_t stream);
 
 cudaError_t launch_combine(const mep_shape_t &s, int32_t H, const mep_plan_t &pl,
                            const uint16_t *y, const float *w, uint16_t *out,

@@ -12,24 +12,29 @@
 // The schedule is the stable sort of (token, k) pairs by (expert, g, k) cut
 // into R chunks of S*K.
 //
-// Structure.  The pairs are split into `nb` contiguous tiles, one per block
-// (nb <= number of SMs, all co-resident), and each tile into 32 contiguous
-// warp ranges.
-//   Phase 1  every warp builds a private histogram of its range in shared
-//            memory (match_any groups equal expert ids, one leader adds the
-//            group size: no atomics); the block turns the 32 warp histograms
-//            into per-warp exclusive offsets and publishes its tile total per
-//            expert to tile[e][b].
+// Structure.  The pairs are split into nt contiguous tiles, each tile into
+// 32 contiguous warp ranges.  With more than one tile the grid is nt + 1
+// co-resident blocks: block 0 is a coordinator that owns no pairs and builds
+// the plan's tables while the others scatter; with one tile a single block
+// does everything and the grid barriers reduce to __syncthreads.
+//   Phase 1  every warp counts its range into a warp-private histogram in
+//            shared memory (shared-memory atomics: only the warp's own lanes
+//            contend) and parks its ids in shared memory; the block turns the
+//            32 warp histograms into per-warp exclusive offsets and publishes
+//            its tile total per expert to tile[e][t].
 //   -- grid barrier --
-//   Phase 2  one warp per expert scans its row tile[e][0..nb) into exclusive
+//   Phase 2  one warp per expert scans its row tile[e][0..nt) into exclusive
 //            per-tile offsets and writes T_e.
 //   -- grid barrier --
-//   Phase 3  every block scans T_e over experts (expert offsets), block 0
-//            writes maxvio, the offsets, segments, CSR pointers and replica
-//            list; every warp walks its range again in (g, k) order and gives
-//            each pair slot = off_e + tile offset + warp offset + rank among
-//            equal ids earlier in the warp (match_any + popc).
-// All the idx reads of phase 3 hit L2 (the plan input is at most a few MB).
+//   Phase 3  every block scans T_e over experts (expert offsets); the
+//            coordinator writes maxvio, the offsets, segments, CSR pointers
+//            and replica list; every tile warp walks its ids again in (g, k)
+//            order and gives each pair slot = off_e + tile offset + warp
+//            offset + rank among equal ids earlier in the warp.  The rank
+//            comes from a peer mask (one ballot per id bit; the lanes holding
+//            the same id) and the popcount of the peers below the lane.
+// A warp whose range exceeds its shared-memory id buffer reads its ids again
+// from global memory (L2 hits) in phase 3.
 #include <climits>
 #include <cstdint>
 
@@ -42,24 +47,45 @@ namespace {
 
 constexpr int kThreads = kPlanThreads;
 constexpr int kWarps = kThreads / 32;
-constexpr int kBatch = 8;  // coalesced 32-pair loads in flight per warp
+constexpr int kBatch = 8;          // 32-pair chunks a warp loads at once
+
+#ifndef MEP_PLAN_PEERS_BALLOT
+#define MEP_PLAN_PEERS_BALLOT 1  // 1: peer masks from bit ballots; 0: match.any
+#endif
 
 struct PlanParams {
   const int32_t *idx;
   int32_t R, S, E, K;
   int64_t NK, SK;
-  int32_t nb;
-  int64_t ppb;  // pairs per tile
+  int32_t nb;    // blocks
+  int32_t nt;    // tiles (nb - 1 with a coordinator, else 1)
+  int64_t ppb;   // pairs per tile
   int32_t full;  // 0: counts + maxvio only
   int32_t *counts, *expert_offset, *slot, *src_pair;
   int4 *seg;
   int32_t *rank_seg_ptr, *expert_seg_ptr, *replica_seg;
   int32_t *num_seg, *num_replicas, *max_count, *status;
   double *maxvio;
-  int32_t *tile;   // workspace [E][nb]
+  int32_t *tile;   // workspace [E][nt]
   uint32_t *bar;   // workspace barrier words
   uint64_t wait_ns;
 };
+
+// Mask of the lanes whose key equals this lane's key; keys are < 2^nbits.
+__device__ __forceinline__ unsigned peers_of(int key, int nbits) {
+#if MEP_PLAN_PEERS_BALLOT
+  unsigned m = 0xffffffffu;
+  for (int b = 0; b < nbits; ++b) {
+    const bool bit = (key >> b) & 1;
+    const unsigned on = __ballot_sync(0xffffffffu, bit);
+    m &= bit ? on : ~on;
+  }
+  return m;
+#else
+  (void)nbits;
+  return __match_any_sync(0xffffffffu, key);
+#endif
+}
 
 // Exclusive prefix sum of one value per thread over the block; *total gets the
 // block sum.  Uses s_w[32]; every thread of the block must call it.
@@ -101,26 +127,41 @@ __device__ __forceinline__ int block_max(int v, int *s_w) {
   return m;
 }
 
+__device__ __forceinline__ bool plan_sync(const PlanParams &p, int k) {
+  if (p.nb == 1) {
+    __syncthreads();
+    return true;
+  }
+  return grid_barrier(p.bar, k * p.nb, p.wait_ns, p.status);
+}
+
 __global__ void __launch_bounds__(kThreads, 1) plan_kernel(PlanParams p) {
-  extern __shared__ int wh_all[];  // [kWarps][E] per-warp histograms / cursors
+  extern __shared__ int smem[];  // [kWarps][E] histograms / cursors, then [kWarps][kPlanIdsPerWarp] ids
   __shared__ int s_w[32];
   __shared__ int s_off[MEP_MAX_EXPERTS + 1];
   __shared__ int s_sbase[MEP_MAX_EXPERTS + 1];
 
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const int E = p.E;
+  const int nbits = 32 - __clz(E);          // 2^nbits > E
+  const int sentinel = (1 << nbits) - 1;    // key of an empty or invalid lane
+  const bool coord = p.nb > 1 && blockIdx.x == 0;
+  const int tile = p.nb > 1 ? (int)blockIdx.x - 1 : 0;
   if (blockIdx.x == 0 && t == 0) *p.status = 0;
 
+  int *wh_all = smem;
   int *wh = wh_all + warp * E;
+  int *ids = smem + kWarps * E + warp * kPlanIdsPerWarp;
   for (int i = t; i < kWarps * E; i += kThreads) wh_all[i] = 0;
   __syncthreads();
 
-  // Tile and warp ranges.
-  const int64_t b0 = (int64_t)blockIdx.x * p.ppb;
-  const int64_t b1 = min(b0 + p.ppb, p.NK);
+  // Tile and warp ranges (the coordinator has none).
+  const int64_t b0 = coord ? 0 : (int64_t)tile * p.ppb;
+  const int64_t b1 = coord ? 0 : min(b0 + p.ppb, p.NK);
   const int64_t n = b1 > b0 ? b1 - b0 : 0;
   const int64_t w0 = b0 + (n * warp) / kWarps;
   const int64_t w1 = b0 + (n * (warp + 1)) / kWarps;
+  const bool keep = (w1 - w0) <= kPlanIdsPerWarp;  // ids stay in shared memory
 
   // ---- phase 1: warp-private histograms ------------------------------------
   bool bad = false;
@@ -129,19 +170,16 @@ __global__ void __launch_bounds__(kThreads, 1) plan_kernel(PlanParams p) {
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
       const int64_t q = c + u * 32 + lane;
-      ev[u] = q < w1 ? __ldg(p.idx + q) : INT_MIN;
+      ev[u] = q < w1 ? __ldg(p.idx + q) : -1;
     }
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
-      if (c + u * 32 >= w1) break;  // warp-uniform
       const int64_t q = c + u * 32 + lane;
-      const bool act = q < w1;
-      const int e = ev[u];
-      const bool valid = act && (unsigned)e < (unsigned)E;
-      bad |= act && !valid;
-      const unsigned peers = __match_any_sync(0xffffffffu, valid ? e : -1);
-      if (valid && lane == __ffs(peers) - 1) wh[e] += __popc(peers);
-      __syncwarp();
+      if (q < w1) {
+        const int e = ev[u];
+        if ((unsigned)e < (unsigned)E) atomicAdd(wh + e, 1); else bad = true;
+        if (keep) ids[q - w0] = e;
+      }
     }
   }
   __syncthreads();
@@ -152,21 +190,29 @@ __global__ void __launch_bounds__(kThreads, 1) plan_kernel(PlanParams p) {
       wh_all[w * E + t] = run;
       run += v;
     }
-    __stcg(p.tile + (int64_t)t * p.nb + blockIdx.x, run);
+    if (!coord) __stcg(p.tile + (int64_t)t * p.nt + tile, run);
   }
   bad = __syncthreads_or(bad);
 
-  if (!grid_barrier(p.bar, p.nb, p.wait_ns, p.status)) return;
+  if (!plan_sync(p, 1)) return;
   if (bad && t == 0) set_status(p.status, MEP_ERR_DEVICE_DATA);
 
   // ---- phase 2: per-expert scan over tiles ----------------------------------
   {
-    const int per = (p.nb + 31) / 32;
+    const int per = (p.nt + 31) / 32;  // tiles per lane, <= 32
     for (int e = blockIdx.x * kWarps + warp; e < E; e += p.nb * kWarps) {
-      int32_t *row = p.tile + (int64_t)e * p.nb;
-      const int lo = min(lane * per, p.nb), hi = min(lo + per, p.nb);
+      int32_t *row = p.tile + (int64_t)e * p.nt;
+      const int lo = min(lane * per, p.nt), hi = min(lo + per, p.nt);
+      int v[8];
       int s = 0;
-      for (int b = lo; b < hi; ++b) s += __ldcg(row + b);
+      if (per <= 8) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] = lo + j < hi ? __ldcg(row + lo + j) : 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) s += v[j];
+      } else {
+        for (int b = lo; b < hi; ++b) s += __ldcg(row + b);
+      }
       int incl = s;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -175,10 +221,20 @@ __global__ void __launch_bounds__(kThreads, 1) plan_kernel(PlanParams p) {
       }
       if (p.full) {
         int run = incl - s;
-        for (int b = lo; b < hi; ++b) {
-          const int v = __ldcg(row + b);
-          __stcg(row + b, run);
-          run += v;
+        if (per <= 8) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            if (lo + j < hi) {
+              __stcg(row + lo + j, run);
+              run += v[j];
+            }
+          }
+        } else {
+          for (int b = lo; b < hi; ++b) {
+            const int x = __ldcg(row + b);
+            __stcg(row + b, run);
+            run += x;
+          }
         }
       }
       const int total = __shfl_sync(0xffffffffu, incl, 31);
@@ -186,7 +242,7 @@ __global__ void __launch_bounds__(kThreads, 1) plan_kernel(PlanParams p) {
     }
   }
 
-  if (!grid_barrier(p.bar, p.nb, p.wait_ns, p.status)) return;
+  if (!plan_sync(p, 2)) return;
 
   // ---- phase 3: offsets, scalars, segments, scatter -------------------------
   const int T = t < E ? __ldcg(p.counts + t) : 0;
@@ -200,9 +256,8 @@ __global__ void __launch_bounds__(kThreads, 1) plan_kernel(PlanParams p) {
       *p.maxvio = (double)((long long)mx * E) / (double)p.NK - 1.0;
     }
   }
-  if (!p.full) return;
 
-  if (blockIdx.x == 0) {
+  if (p.full && blockIdx.x == 0) {  // the coordinator (or the only block)
     const int64_t SK = p.SK;
     int nseg_e = 0, r0 = 0, r1 = -1;
     if (t < E && T > 0) {
@@ -254,29 +309,22 @@ __global__ void __launch_bounds__(kThreads, 1) plan_kernel(PlanParams p) {
     }
   }
 
-  // Per-warp cursors: expert offset + tile offset + warp offset.
-  if (t < E) {
-    const int base = off + __ldcg(p.tile + (int64_t)t * p.nb + blockIdx.x);
-    for (int w = 0; w < kWarps; ++w) wh_all[w * E + t] += base;
-  }
-  __syncthreads();
-
-  const unsigned lt = lanemask_lt();
-  for (int64_t c = w0; c < w1; c += 32 * kBatch) {
-    int ev[kBatch];
-#pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      const int64_t q = c + u * 32 + lane;
-      ev[u] = q < w1 ? __ldg(p.idx + q) : INT_MIN;
+  if (p.full && !coord) {
+    // Per-warp cursors: expert offset + tile offset + warp offset.
+    if (t < E) {
+      const int base = off + __ldcg(p.tile + (int64_t)t * p.nt + tile);
+      for (int w = 0; w < kWarps; ++w) wh_all[w * E + t] += base;
     }
-#pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      if (c + u * 32 >= w1) break;
-      const int64_t q = c + u * 32 + lane;
+    __syncthreads();
+
+    const unsigned lt = lanemask_lt();
+    for (int64_t c = w0; c < w1; c += 32) {
+      const int64_t q = c + lane;
       const bool act = q < w1;
-      const int e = ev[u];
-      const bool valid = act && (unsigned)e < (unsigned)E;
-      const unsigned peers = __match_any_sync(0xffffffffu, valid ? e : -1);
+      int e = -1;
+      if (act) e = keep ? ids[q - w0] : __ldg(p.idx + q);
+      const bool valid = (unsigned)e < (unsigned)E;
+      const unsigned peers = peers_of(valid ? e : sentinel, nbits);
       const int base = valid ? wh[e] : 0;
       __syncwarp();
       if (valid) {
@@ -290,6 +338,7 @@ __global__ void __launch_bounds__(kThreads, 1) plan_kernel(PlanParams p) {
       __syncwarp();
     }
   }
+  if (p.nb > 1) grid_barrier_exit(p.bar, p.nb);
 }
 
 struct PlanDev {
@@ -313,7 +362,7 @@ cudaError_t launch_plan(const mep_shape_t &s, const int32_t *idx, const mep_plan
   if (err != cudaSuccess) return err;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   PlanDev &d = g_plan_dev[dev];
-  const size_t smem = (size_t)kWarps * s.E * sizeof(int);
+  const size_t smem = ((size_t)kWarps * s.E + (size_t)kWarps * kPlanIdsPerWarp) * sizeof(int);
   if (d.smem_attr != (int)smem) {
     err = cudaFuncSetAttribute(plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
@@ -328,15 +377,18 @@ cudaError_t launch_plan(const mep_shape_t &s, const int32_t *idx, const mep_plan
   }
   const int64_t NK = (int64_t)s.R * s.S * s.K;
   int64_t want = (NK + kPlanMinPairsPerBlock - 1) / kPlanMinPairsPerBlock;
-  int nb = (int)std::min<int64_t>(std::max<int64_t>(want, 1),
-                                  std::min(d.max_blocks, kPlanMaxBlocks));
+  // One block for a single tile; otherwise a coordinator plus nt tiles.
+  const int64_t cap = std::min(d.max_blocks, kPlanMaxBlocks) - 1;
+  const int nt = (int)std::max<int64_t>(1, std::min<int64_t>(want, cap));
+  const int nb = nt > 1 ? nt + 1 : 1;
   PlanParams p{};
   p.idx = idx;
   p.R = s.R; p.S = s.S; p.E = s.E; p.K = s.K;
   p.NK = NK;
   p.SK = (int64_t)s.S * s.K;
   p.nb = nb;
-  p.ppb = (NK + nb - 1) / nb;
+  p.nt = nt;
+  p.ppb = (NK + nt - 1) / nt;
   p.full = full;
   p.counts = pl.counts; p.expert_offset = pl.expert_offset; p.slot = pl.slot;
   p.src_pair = pl.src_pair; p.seg = reinterpret_cast<int4 *>(pl.seg);

@@ -26,7 +26,7 @@
 #define MEP_REDUCE_U 4
 #endif
 #ifndef MEP_REDUCE_BLOCKS_PER_SM
-#define MEP_REDUCE_BLOCKS_PER_SM 16
+#define MEP_REDUCE_BLOCKS_PER_SM 1024
 #endif
 #ifndef MEP_REDUCE_MIN_BLOCKS
 #define MEP_REDUCE_MIN_BLOCKS 3  // launch bound: resident blocks per SM
