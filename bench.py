@@ -11,7 +11,9 @@ mep_dispatch -> mep_combine -> mep_reduce_replica_grads, all through the C ABI.
   device time), inputs resident in HBM, L2 flushed (512 MB write) between
   steps outside the timed events.
 * e2e: the same metric through the public API with pinned host buffers: every
-  step copies that step's inputs host->device and the outputs back.
+  step copies that step's inputs host->device and its outputs (combine
+  output, home gradients, plan scalars) back; consecutive steps overlap on
+  separate copy and compute streams.
 * roofline: the step's dominant kernel, algorithmic bytes / its mean event
   time, against the measured HBM copy peak.
 * cpu_baseline / --impl reference: the CPU oracle, single-threaded, on a
@@ -57,7 +59,7 @@ def parse_args():
                     help="tokens per rank (default: the workload's); for small profiling cases")
     ap.add_argument("--P", type=int, default=None,
                     help="gradient row length (default: the workload's); for small profiling cases")
-    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--e2e-steps", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle baseline sample")
@@ -352,7 +354,10 @@ def main():
                 "frac": kernels[dom]["gbs"] / peak, "traffic": dram_traffic(dom, wl.name),
                 "kernel": dom, "peak_source": f"{peak_kind} hbm_gbs (copy)"}
 
-    # ---- e2e: host buffers through the public API
+    # ---- e2e: host buffers through the public API, as a user would pipeline
+    # it: two device buffer sets, inputs copied host->device on one stream,
+    # the path on another, outputs copied back on a third, so the two copy
+    # directions and the kernels overlap across consecutive steps.
     e2e = None
     if args.e2e_steps > 0:
         pin = dict(pin_memory=True)
@@ -361,43 +366,76 @@ def main():
         hx = torch.empty(x.shape, dtype=x.dtype, **pin).copy_(x)
         hy = torch.empty(y.shape, dtype=y.dtype, **pin).copy_(y)
         hG = torch.empty(G.shape, dtype=G.dtype, **pin).copy_(G) if P else None
-        ho = torch.empty(out.shape, dtype=out.dtype, **pin)
-        hh = torch.empty(home.shape, dtype=home.dtype, **pin) if P else None
-        hsc = torch.empty(4, dtype=torch.int32, **pin)
-        hmv = torch.empty(1, dtype=torch.float64, **pin)
+        sets = []
+        for b in range(2):
+            d = dict(idx=idx if b == 0 else torch.empty_like(idx), w=w if b == 0 else torch.empty_like(w),
+                     x=x if b == 0 else torch.empty_like(x), y=y if b == 0 else torch.empty_like(y),
+                     G=(G if b == 0 else torch.empty_like(G)) if P else None,
+                     plan=plan if b == 0 else mep.Plan(s, dev),
+                     buf=buf if b == 0 else torch.empty_like(buf),
+                     out=out if b == 0 else torch.empty_like(out),
+                     home=(home if b == 0 else torch.empty_like(home)) if P else None,
+                     ho=torch.empty(out.shape, dtype=out.dtype, **pin),
+                     hh=torch.empty(home.shape, dtype=home.dtype, **pin) if P else None,
+                     hsc=torch.empty(4, dtype=torch.int32, **pin),
+                     hmv=torch.empty(1, dtype=torch.float64, **pin))
+            d["ev_in"], d["ev_cmp"], d["ev_out"] = (torch.cuda.Event() for _ in range(3))
+            sets.append(d)
         h2d = sum(t.numel() * t.element_size() for t in (hi, hw, hx, hy) + ((hG,) if P else ()))
-        d2h = sum(t.numel() * t.element_size() for t in (ho, hsc, hmv) + ((hh,) if P else ()))
+        d2h = sum(t.numel() * t.element_size()
+                  for t in (sets[0]["ho"], sets[0]["hsc"], sets[0]["hmv"]) + ((sets[0]["hh"],) if P else ()))
+        s_in, s_cmp, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
 
-        def e2e_step():
-            idx.copy_(hi, non_blocking=True)
-            w.copy_(hw, non_blocking=True)
-            x.copy_(hx, non_blocking=True)
-            y.copy_(hy, non_blocking=True)
-            if P:
-                G.copy_(hG, non_blocking=True)
-            step()
-            ho.copy_(out, non_blocking=True)
-            if P:
-                hh.copy_(home, non_blocking=True)
-            hsc.copy_(plan.scalars, non_blocking=True)
-            hmv.copy_(plan.maxvio_t, non_blocking=True)
+        def e2e_step(i):
+            d = sets[i % 2]
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(d["ev_cmp"])      # step i-2 has finished reading these inputs
+                d["idx"].copy_(hi, non_blocking=True)
+                d["w"].copy_(hw, non_blocking=True)
+                d["x"].copy_(hx, non_blocking=True)
+                d["y"].copy_(hy, non_blocking=True)
+                if P:
+                    d["G"].copy_(hG, non_blocking=True)
+                d["ev_in"].record(s_in)
+            with torch.cuda.stream(s_cmp):
+                s_cmp.wait_event(d["ev_in"])
+                if i >= 2:
+                    s_cmp.wait_event(d["ev_out"])     # step i-2's outputs are on the host
+                pl = d["plan"]
+                mep.mep_plan(s, d["idx"], pl)
+                mep.mep_dispatch(s, H, pl, d["x"], d["buf"])
+                mep.mep_combine(s, H, pl, d["y"], d["w"], d["out"])
+                if P:
+                    mep.mep_reduce_replica_grads(s, pl, P, d["G"], d["home"])
+                d["ev_cmp"].record(s_cmp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(d["ev_cmp"])
+                d["ho"].copy_(d["out"], non_blocking=True)
+                if P:
+                    d["hh"].copy_(d["home"], non_blocking=True)
+                d["hsc"].copy_(d["plan"].scalars, non_blocking=True)
+                d["hmv"].copy_(d["plan"].maxvio_t, non_blocking=True)
+                d["ev_out"].record(s_out)
 
-        e2e_step()
+        for i in range(2):
+            e2e_step(i)
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         torch.cuda.synchronize()
-        e0.record()
-        for _ in range(args.e2e_steps):
-            e2e_step()
-        e1.record()
+        e0.record(s_in)
+        for i in range(2, 2 + args.e2e_steps):
+            e2e_step(i)
+        e1.record(s_out)
         torch.cuda.synchronize()
         ms_e2e = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, world, dev)
-        if int(hsc[3].item()) != 0:
+        if any(int(d["hsc"][3].item()) != 0 for d in sets):
             raise RuntimeError("device status not OK after e2e steps")
         e2e = {"value": whole_job_rate(N, world, ms_e2e), "unit": "tokens/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e}
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e,
+               "pipeline": "2 buffer sets; H2D, kernels, D2H on 3 streams"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
