@@ -79,6 +79,12 @@ class Oracle:
         L.ora_combine.restype = None
         L.ora_reduce.argtypes = [ctypes.c_int, _i32p, ctypes.c_int64, _f32p, _f64p, _f64p]
         L.ora_reduce.restype = None
+        L.ora_combine_backward.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int64, _i32p, _f32p,
+                                           _u16p, _u16p, _u16p, _f64p, _f64p, _f64p]
+        L.ora_combine_backward.restype = None
+        L.ora_dispatch_backward.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int64, _i32p, _u16p,
+                                            _u16p, _f64p, _f64p]
+        L.ora_dispatch_backward.restype = None
         self.lib = L
 
     # -- scalars -----------------------------------------------------------
@@ -165,6 +171,43 @@ class Oracle:
         absum = np.empty((E, P), np.float64)
         self.lib.ora_reduce(E, _p(ptr, _i32p), P, _p(G, _f32p), _p(home, _f64p), _p(absum, _f64p))
         return home, absum
+
+    # -- backward of combine and dispatch --------------------------------------
+    def combine_backward(self, slot, w, grad_out, y):
+        """``slot`` int32 ``[n, K]`` (rows of ``y``), ``w`` float32 ``[n, K]``,
+        ``grad_out`` bf16-as-uint16 ``[n, H]``, ``y`` ``[rows, H]``.  Returns
+        (grad_y bf16 ``[rows, H]`` -- rows not named by ``slot`` stay zero --,
+        its unrounded binary64 values, grad_w binary64 ``[n, K]``, sum of
+        |terms| of each dot product)."""
+        slot = np.ascontiguousarray(slot, dtype=np.int32)
+        w = np.ascontiguousarray(w, dtype=np.float32)
+        go = np.ascontiguousarray(grad_out, dtype=np.uint16)
+        y = np.ascontiguousarray(y, dtype=np.uint16)
+        n, K = slot.shape
+        H = go.shape[1]
+        gy = np.zeros((y.shape[0], H), np.uint16)
+        gye = np.zeros((y.shape[0], H), np.float64)
+        gw = np.empty((n, K), np.float64)
+        gwa = np.empty((n, K), np.float64)
+        self.lib.ora_combine_backward(n, K, H, _p(slot, _i32p), _p(w, _f32p), _p(go, _u16p),
+                                      _p(y, _u16p), _p(gy, _u16p), _p(gye, _f64p), _p(gw, _f64p),
+                                      _p(gwa, _f64p))
+        return gy, gye, gw, gwa
+
+    def dispatch_backward(self, slot, grad_buf):
+        """``slot`` int32 ``[n, K]`` (rows of ``grad_buf``), ``grad_buf``
+        bf16-as-uint16 ``[rows, H]``; returns (grad_x bf16 ``[n, H]``, binary64
+        sum, sum of |terms|)."""
+        slot = np.ascontiguousarray(slot, dtype=np.int32)
+        gb = np.ascontiguousarray(grad_buf, dtype=np.uint16)
+        n, K = slot.shape
+        H = gb.shape[1]
+        gx = np.empty((n, H), np.uint16)
+        ex = np.empty((n, H), np.float64)
+        ab = np.empty((n, H), np.float64)
+        self.lib.ora_dispatch_backward(n, K, H, _p(slot, _i32p), _p(gb, _u16p), _p(gx, _u16p),
+                                       _p(ex, _f64p), _p(ab, _f64p))
+        return gx, ex, ab
 
 
 _default: Oracle | None = None

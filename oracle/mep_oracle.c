@@ -33,7 +33,11 @@
  * of S*K slots; home(e) = e / (E/R); a (rank, expert) segment whose rank is
  * not home(e) is a replica; combine is the K-term weighted sum back to token
  * order; the replica reduction sums an expert's segment rows in ascending
- * segment order.
+ * segment order.  The backward of dispatch and combine (the training step's
+ * return path, [P1-how]: a backward pass exists) is the adjoint of the
+ * forward maps: combine's gradient flows to each slot weighted by its router
+ * weight, and to each router weight as a dot product with the slot's expert
+ * output; dispatch's gradient is the sum of the K slot gradients of a token.
  */
 #include <math.h>
 #include <stddef.h>
@@ -284,6 +288,64 @@ void ora_reduce(int E, const int32_t *expert_seg_ptr, int64_t P,
             home[(int64_t)e * P + i] = acc;
             if (absum)
                 absum[(int64_t)e * P + i] = mag;
+        }
+    }
+}
+
+/* ---- backward of combine (adjoint of ora_combine) ----------------------- *
+ * For out[g] = sum_k w[g,k] * y[slot[g,k]]:
+ *   grad_y[slot[g,k], h] = bf16( w[g,k] * grad_out[g, h] )     (one rounding)
+ *   grad_w[g, k]         = sum_h grad_out[g, h] * y[slot[g,k], h]  (binary64)
+ * grad_y has one row per slot; every slot belongs to exactly one (g, k).
+ * gy_exact / gw_absum (may be NULL) receive the unrounded product and the
+ * sum of |terms| of each dot product, for error bounds. */
+void ora_combine_backward(int64_t ntok, int K, int64_t H, const int32_t *slot,
+                          const float *w, const uint16_t *grad_out,
+                          const uint16_t *y, uint16_t *grad_y, double *gy_exact,
+                          double *grad_w, double *gw_absum)
+{
+    for (int64_t g = 0; g < ntok; ++g) {
+        for (int k = 0; k < K; ++k) {
+            int64_t p = slot[g * K + k];
+            double wk = (double)w[g * K + k];
+            double dot = 0.0, mag = 0.0;
+            for (int64_t h = 0; h < H; ++h) {
+                double go = (double)ora_bf16_to_f32(grad_out[g * H + h]);
+                double prod = wk * go;                 /* exact in binary64 */
+                grad_y[p * H + h] = ora_f64_to_bf16(prod);
+                if (gy_exact)
+                    gy_exact[p * H + h] = prod;
+                double term = go * (double)ora_bf16_to_f32(y[p * H + h]);  /* exact */
+                dot += term;
+                mag += fabs(term);
+            }
+            grad_w[g * K + k] = dot;
+            if (gw_absum)
+                gw_absum[g * K + k] = mag;
+        }
+    }
+}
+
+/* ---- backward of dispatch (adjoint of ora_dispatch) --------------------- *
+ * For buf[slot[g,k]] = x[g]:  grad_x[g, h] = bf16( sum_k grad_buf[slot[g,k], h] ),
+ * summed in binary64 and rounded once.  exact / absum as in ora_combine. */
+void ora_dispatch_backward(int64_t ntok, int K, int64_t H, const int32_t *slot,
+                           const uint16_t *grad_buf, uint16_t *grad_x,
+                           double *exact, double *absum)
+{
+    for (int64_t g = 0; g < ntok; ++g) {
+        for (int64_t h = 0; h < H; ++h) {
+            double acc = 0.0, mag = 0.0;
+            for (int k = 0; k < K; ++k) {
+                double v = (double)ora_bf16_to_f32(grad_buf[(int64_t)slot[g * K + k] * H + h]);
+                acc += v;
+                mag += fabs(v);
+            }
+            grad_x[g * H + h] = ora_f64_to_bf16(acc);
+            if (exact)
+                exact[g * H + h] = acc;
+            if (absum)
+                absum[g * H + h] = mag;
         }
     }
 }

@@ -394,6 +394,79 @@ def pin_reduce(ora):
             assert abs(Fraction(home[e, i]) - v) <= Fraction(8, 2 ** 52) * max(1, abs(v))
 
 
+# ------------------------------------------------------------- backward
+
+def _bf16_rows(ora, rng, rows, H, scale=1.0):
+    return np.array([[ora.f64_to_bf16(float(v)) for v in r]
+                     for r in rng.standard_normal((rows, H)) * scale], np.uint16)
+
+
+def _perm_slots(rng, n, K):
+    """A slot table like a plan's: every row of a [n*K, H] buffer used once."""
+    return rng.permutation(n * K).astype(np.int32).reshape(n, K)
+
+
+def pin_combine_backward(ora):
+    rng = np.random.default_rng(21)
+    for K in (1, 2, 5, 16):
+        n, H = 4, 8
+        slot = _perm_slots(rng, n, K)
+        w = rng.random((n, K)).astype(np.float32)
+        y = _bf16_rows(ora, rng, n * K, H)
+        go = _bf16_rows(ora, rng, n, H)
+        gy, gye, gw, gwa = ora.combine_backward(slot, w, go, y)
+        F = lambda b: Fraction(_bits_to_f32(int(b)))
+        # adjoint: <combine(y), go> == <y, grad_y>, exactly
+        lhs = sum((F(go[g, h]) * Fraction(float(w[g, k])) * F(y[slot[g, k], h])
+                   for g in range(n) for h in range(H) for k in range(K)), Fraction(0))
+        rhs = sum((F(y[p, h]) * Fraction(gye[p, h]) for p in range(n * K) for h in range(H)),
+                  Fraction(0))
+        assert lhs == rhs, (K, float(lhs), float(rhs))
+        for g in range(n):
+            for k in range(K):
+                p = slot[g, k]
+                for h in range(H):
+                    want = Fraction(float(w[g, k])) * F(go[g, h])
+                    assert Fraction(gye[p, h]) == want
+                    assert gy[p, h] == bf16_round_by_search(float(want))
+                dot = sum((F(go[g, h]) * F(y[p, h]) for h in range(H)), Fraction(0))
+                assert abs(Fraction(gw[g, k]) - dot) <= Fraction(H, 2 ** 52) * Fraction(gwa[g, k])
+    # unit weight, K = 1: the slot gradient is the output gradient itself
+    slot = np.arange(6, dtype=np.int32).reshape(6, 1)
+    go = _bf16_rows(ora, rng, 6, 8)
+    gy, _, _, _ = ora.combine_backward(slot, np.ones((6, 1), np.float32), go, go)
+    assert np.array_equal(gy, go)
+
+
+def pin_dispatch_backward(ora):
+    rng = np.random.default_rng(22)
+    F = lambda b: Fraction(_bits_to_f32(int(b)))
+    for K in (1, 3, 16):
+        n, H = 5, 8
+        slot = _perm_slots(rng, n, K)
+        x = _bf16_rows(ora, rng, n, H)
+        gb = _bf16_rows(ora, rng, n * K, H)
+        gx, ex, ab = ora.dispatch_backward(slot, gb)
+        # adjoint: <dispatch(x), grad_buf> == <x, grad_x_exact>
+        src = np.empty(n * K, np.int32)
+        src[slot.reshape(-1)] = np.arange(n * K, dtype=np.int32)
+        buf = ora.dispatch(K, src, x)
+        lhs = sum((F(buf[p, h]) * F(gb[p, h]) for p in range(n * K) for h in range(H)), Fraction(0))
+        rhs = sum((F(x[g, h]) * Fraction(ex[g, h]) for g in range(n) for h in range(H)), Fraction(0))
+        assert lhs == rhs
+        for g in range(n):
+            for h in range(H):
+                v = sum((F(gb[slot[g, k], h]) for k in range(K)), Fraction(0))
+                assert Fraction(ex[g, h]) == v
+                assert gx[g, h] == bf16_round_by_search(float(v))
+    # rows of constant value c_p: grad_x[g] = sum_k c_{slot[g,k]}
+    n, K, H = 3, 4, 8
+    slot = _perm_slots(rng, n, K)
+    gb = np.array([[ora.f64_to_bf16(float(p + 1))] * H for p in range(n * K)], np.uint16)
+    gx, ex, _ = ora.dispatch_backward(slot, gb)
+    assert np.array_equal(ex, np.repeat((slot + 1).sum(axis=1, keepdims=True).astype(np.float64), H, axis=1))
+
+
 ALL_PINS = [pin_bf16_widen, pin_bf16_rounding, pin_plan_golden, pin_plan_bruteforce,
             pin_plan_invariants, pin_closed_forms, pin_errors, pin_dispatch,
-            pin_combine, pin_reduce]
+            pin_combine, pin_reduce, pin_combine_backward, pin_dispatch_backward]

@@ -54,6 +54,17 @@ MUTANTS = {
     "reduce_uses_next_expert": (
         "for (int32_t s = expert_seg_ptr[e]; s < expert_seg_ptr[e + 1]; ++s)",
         "for (int32_t s = expert_seg_ptr[e]; s < expert_seg_ptr[e + 1] && e + 1 < E; ++s)"),
+    "combine_bwd_first_weight_only": (
+        "double wk = (double)w[g * K + k];", "double wk = (double)w[g * K];"),
+    "combine_bwd_gradw_uses_grad_out_twice": (
+        "double term = go * (double)ora_bf16_to_f32(y[p * H + h]);  /* exact */",
+        "double term = go * go;"),
+    "combine_bwd_row_by_pair_not_slot": (
+        "grad_y[p * H + h] = ora_f64_to_bf16(prod);",
+        "grad_y[(g * K + k) * H + h] = ora_f64_to_bf16(prod);"),
+    "dispatch_bwd_drops_last_k": (
+        "for (int k = 0; k < K; ++k) {\n                double v = (double)ora_bf16_to_f32(grad_buf",
+        "for (int k = 0; k < K - 1; ++k) {\n                double v = (double)ora_bf16_to_f32(grad_buf"),
 }
 
 
