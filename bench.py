@@ -61,6 +61,8 @@ def parse_args():
                     help="gradient row length (default: the workload's); for small profiling cases")
     ap.add_argument("--e2e-steps", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-backward", action="store_true",
+                    help="skip the separately timed backward kernels")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle baseline sample")
     return ap.parse_args()
@@ -354,6 +356,35 @@ def main():
                 "frac": kernels[dom]["gbs"] / peak, "traffic": dram_traffic(dom, wl.name),
                 "kernel": dom, "peak_source": f"{peak_kind} hbm_gbs (copy)"}
 
+    # ---- backward of combine and dispatch (timed alone, not part of the step)
+    backward = None
+    if not args.no_backward:
+        grad_y = torch.empty_like(buf)
+        grad_w = torch.empty((N, K), dtype=torch.float32, device=dev)
+        grad_x = torch.empty_like(x)
+        bwd = {"combine_backward": (lambda: mep.mep_combine_backward(s, H, plan, out, w, y, grad_y, grad_w),
+                                    N * H * 2 + 2 * NK * H * 2 + NK * 8),
+               "dispatch_backward": (lambda: mep.mep_dispatch_backward(s, H, plan, buf, grad_x),
+                                     NK * H * 2 + N * H * 2 + NK * 4)}
+        backward = {}
+        for name, (fn, nbytes) in bwd.items():
+            ts = []
+            for it in range(3 + 20):
+                flush.zero_()
+                b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                b0.record()
+                fn()
+                b1.record()
+                if it >= 3:
+                    torch.cuda.synchronize()
+                    ts.append(b0.elapsed_time(b1))
+            ms = float(np.median(ts))
+            gbs = nbytes / (ms * 1e-3) / 1e9
+            backward[name] = {"ms": ms, "bytes": nbytes, "gbs": gbs, "frac": gbs / peak}
+        if mep.mep_read_status(plan) != 0:
+            raise RuntimeError("device status not OK after the backward kernels")
+        del grad_y, grad_w, grad_x
+
     # ---- e2e: host buffers through the public API, as a user would pipeline
     # it: two device buffer sets, inputs copied host->device on one stream,
     # the path on another, outputs copied back on a third, so the two copy
@@ -460,6 +491,7 @@ def main():
             "clocks": clocks,
             "gpu_launches": launches_per_step * args.steps,
             "stages_ms": stage_ms,
+            "backward_kernels": backward,
             "kernels": kernels,
             "plan_us": stage_ms["plan"] * 1e3,
             "pdc_tokens_per_s": whole_job_rate(N, world, pdc_ms),

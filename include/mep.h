@@ -178,6 +178,30 @@ MEP_API mep_status_t mep_reduce_replica_grads(mep_shape_t shape, const mep_plan_
                                       int64_t P, const float *seg_grads,
                                       float *home_grads, void *stream);
 
+/* Backward of mep_combine (the adjoint of the weighted combine; the backward
+ * pass of "How MoonEP works").
+ *   grad_out bf16 [N, H]        gradient of the combine output.
+ *   topk_w   float32 [N, K]     router weights of the forward combine.
+ *   y        bf16 [R, S*K, H]   expert outputs the forward combine read.
+ *   grad_y   bf16 [R, S*K, H] out: grad_y[slot[g,k], :] = w[g,k] * grad_out[g, :],
+ *            rounded once to nearest-even bf16 (every slot is written once).
+ *   grad_w   float32 [N, K] out: grad_w[g,k] = sum_h grad_out[g,h] * y[slot[g,k],h],
+ *            float32 FMAs per lane, then a fixed-order warp reduction.
+ * Row buffers 16-byte aligned, H % 8 == 0. */
+MEP_API mep_status_t mep_combine_backward(mep_shape_t shape, int32_t H, const mep_plan_t *plan,
+                                          const uint16_t *grad_out, const float *topk_w,
+                                          const uint16_t *y, uint16_t *grad_y, float *grad_w,
+                                          void *stream);
+
+/* Backward of mep_dispatch (the adjoint of the copy into the slots).
+ *   grad_buf bf16 [R, S*K, H]   gradient of the dispatch buffer.
+ *   grad_x   bf16 [N, H] out: grad_x[g,:] = bf16_rne(sum over k = 0..K-1, in
+ *            that order, of grad_buf[slot[g,k], :]), accumulated in float32.
+ * Row buffers 16-byte aligned, H % 8 == 0. */
+MEP_API mep_status_t mep_dispatch_backward(mep_shape_t shape, int32_t H, const mep_plan_t *plan,
+                                           const uint16_t *grad_buf, uint16_t *grad_x,
+                                           void *stream);
+
 /* mep_plan without a caller-supplied workspace, for callers that cannot
  * allocate device memory (no allocator in their runtime, or a host framework
  * that owns the device memory pool and forbids allocation after start-up).

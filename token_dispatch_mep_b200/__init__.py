@@ -19,7 +19,7 @@ import torch
 __all__ = [
     "MepError", "Shape", "Plan", "load_library", "library_path",
     "mep_plan_workspace_bytes", "mep_maxvio", "mep_plan", "mep_plan_noalloc", "mep_dispatch",
-    "mep_combine",
+    "mep_combine", "mep_combine_backward", "mep_dispatch_backward",
     "mep_reduce_replica_grads", "mep_read_status", "mep_status_string",
     "mep_set_wait_limit_ns", "mep_get_wait_limit_ns", "mep_version", "STATUS",
 ]
@@ -34,7 +34,7 @@ STATUS = {0: "MEP_OK", 1: "MEP_ERR_INVALID_ARG", 2: "MEP_ERR_MISALIGNED", 3: "ME
 ABI_SYMBOLS = ("mep_plan_workspace_bytes", "mep_maxvio", "mep_plan", "mep_dispatch", "mep_combine",
                "mep_reduce_replica_grads", "mep_read_status", "mep_status_string",
                "mep_set_wait_limit_ns", "mep_get_wait_limit_ns", "mep_version",
-               "mep_plan_noalloc")
+               "mep_plan_noalloc", "mep_combine_backward", "mep_dispatch_backward")
 
 
 class MepError(RuntimeError):
@@ -106,6 +106,8 @@ def load_library():
         "mep_get_wait_limit_ns": ([], u64),
         "mep_version": ([], i32),
         "mep_plan_noalloc": ([Shape, vp, P, vp], ctypes.c_int),
+        "mep_combine_backward": ([Shape, i32, P, vp, vp, vp, vp, vp, vp], ctypes.c_int),
+        "mep_dispatch_backward": ([Shape, i32, P, vp, vp, vp], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -253,6 +255,30 @@ def mep_combine(shape, H: int, plan: Plan, y, topk_w, out):
     wp = _need(topk_w, "topk_w", torch.float32, s.NK, dev)
     op = _need(out, "out", torch.bfloat16, s.N * H, dev)
     _ok(L.mep_combine(s, int(H), ctypes.byref(plan.struct), yp, wp, op, _stream(dev)), "mep_combine")
+
+
+def mep_combine_backward(shape, H: int, plan: Plan, grad_out, topk_w, y, grad_y, grad_w):
+    """Adjoint of mep_combine: ``grad_y[slot[g,k]] = bf16(w[g,k] * grad_out[g])``,
+    ``grad_w[g,k] = <grad_out[g], y[slot[g,k]]>``."""
+    L, s = load_library(), _shape(shape)
+    dev = plan.device
+    args = [_need(grad_out, "grad_out", torch.bfloat16, s.N * H, dev),
+            _need(topk_w, "topk_w", torch.float32, s.NK, dev),
+            _need(y, "y", torch.bfloat16, s.NK * H, dev),
+            _need(grad_y, "grad_y", torch.bfloat16, s.NK * H, dev),
+            _need(grad_w, "grad_w", torch.float32, s.NK, dev)]
+    _ok(L.mep_combine_backward(s, int(H), ctypes.byref(plan.struct), *args, _stream(dev)),
+        "mep_combine_backward")
+
+
+def mep_dispatch_backward(shape, H: int, plan: Plan, grad_buf, grad_x):
+    """Adjoint of mep_dispatch: ``grad_x[g] = bf16(sum_k grad_buf[slot[g,k]])``."""
+    L, s = load_library(), _shape(shape)
+    dev = plan.device
+    gb = _need(grad_buf, "grad_buf", torch.bfloat16, s.NK * H, dev)
+    gx = _need(grad_x, "grad_x", torch.bfloat16, s.N * H, dev)
+    _ok(L.mep_dispatch_backward(s, int(H), ctypes.byref(plan.struct), gb, gx, _stream(dev)),
+        "mep_dispatch_backward")
 
 
 def mep_reduce_replica_grads(shape, plan: Plan, P: int, seg_grads, home_grads):

@@ -123,6 +123,32 @@ mep_status_t mep_reduce_replica_grads(mep_shape_t shape, const mep_plan_t *plan,
   return from_cuda(mep::launch_reduce(shape, *plan, P, seg_grads, home_grads, as_stream(stream)));
 }
 
+mep_status_t mep_combine_backward(mep_shape_t shape, int32_t H, const mep_plan_t *plan,
+                                  const uint16_t *grad_out, const float *topk_w, const uint16_t *y,
+                                  uint16_t *grad_y, float *grad_w, void *stream) {
+  mep_status_t st = check_shape(shape);
+  if (st != MEP_OK) return st;
+  if ((st = check_hidden(H)) != MEP_OK) return st;
+  if (!plan || !plan->slot || !plan->status || !grad_out || !topk_w || !y || !grad_y || !grad_w)
+    return MEP_ERR_INVALID_ARG;
+  if (!aligned(grad_out, 16) || !aligned(y, 16) || !aligned(grad_y, 16) || !aligned(topk_w, 4) ||
+      !aligned(grad_w, 4) || !aligned(plan->slot, 4))
+    return MEP_ERR_MISALIGNED;
+  return from_cuda(mep::launch_combine_backward(shape, H, *plan, grad_out, topk_w, y, grad_y,
+                                                grad_w, as_stream(stream)));
+}
+
+mep_status_t mep_dispatch_backward(mep_shape_t shape, int32_t H, const mep_plan_t *plan,
+                                   const uint16_t *grad_buf, uint16_t *grad_x, void *stream) {
+  mep_status_t st = check_shape(shape);
+  if (st != MEP_OK) return st;
+  if ((st = check_hidden(H)) != MEP_OK) return st;
+  if (!plan || !plan->slot || !plan->status || !grad_buf || !grad_x) return MEP_ERR_INVALID_ARG;
+  if (!aligned(grad_buf, 16) || !aligned(grad_x, 16) || !aligned(plan->slot, 4))
+    return MEP_ERR_MISALIGNED;
+  return from_cuda(mep::launch_combine(shape, H, *plan, grad_buf, nullptr, grad_x, as_stream(stream)));
+}
+
 mep_status_t mep_read_status(const mep_plan_t *plan, void *stream) {
   if (!plan || !plan->status) return MEP_ERR_INVALID_ARG;
   int32_t host = 0;

@@ -14,6 +14,10 @@
 // overlap.  Each lane then issues all K x kU independent 16-byte streaming
 // loads before it touches any of them, adds them in k order with float32
 // FMAs, rounds to bf16 and writes 16 bytes per chunk (streaming store).
+//
+// With no weights (w == nullptr) every weight is 1 and the kernel is the
+// backward of dispatch: grad_x[g] = bf16(sum_k grad_buf[slot[g,k]]) (an FMA
+// with weight 1 rounds exactly like an addition).
 #include <algorithm>
 #include <cstdint>
 
@@ -90,7 +94,7 @@ __global__ void __launch_bounds__(kThreads, MEP_COMBINE_MIN_BLOCKS) combine_kern
     if (t < ntask && lane < p.K) {
       const int64_t g = t / p.parts;
       sl = __ldg(p.slot + g * p.K + lane);
-      wt = __ldg(p.w + g * p.K + lane);
+      wt = p.w != nullptr ? __ldg(p.w + g * p.K + lane) : 1.f;
     }
   };
   int sl, nsl;
