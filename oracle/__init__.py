@@ -85,6 +85,9 @@ class Oracle:
         L.ora_dispatch_backward.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int64, _i32p, _u16p,
                                             _u16p, _f64p, _f64p]
         L.ora_dispatch_backward.restype = None
+        L.ora_prefetch_replicas.argtypes = [ctypes.c_int32, _i32p, _i32p, ctypes.c_int64,
+                                            ctypes.c_void_p, ctypes.c_void_p]
+        L.ora_prefetch_replicas.restype = None
         self.lib = L
 
     # -- scalars -----------------------------------------------------------
@@ -208,6 +211,21 @@ class Oracle:
         self.lib.ora_dispatch_backward(n, K, H, _p(slot, _i32p), _p(gb, _u16p), _p(gx, _u16p),
                                        _p(ex, _f64p), _p(ab, _f64p))
         return gx, ex, ab
+
+    # -- replica weight prefetch -------------------------------------------
+    def prefetch_replicas(self, plan: dict, w_home: np.ndarray) -> np.ndarray:
+        """Rows ``w_rep[j] = w_home[expert of replica j]`` for the plan's
+        replicas (``w_home`` any dtype, ``[E, ...]``)."""
+        w_home = np.ascontiguousarray(w_home)
+        nr = int(plan["num_replicas"])
+        rep = np.ascontiguousarray(plan["replica_seg"], dtype=np.int32)
+        seg = np.ascontiguousarray(plan["seg"], dtype=np.int32)
+        row = w_home[0].nbytes if w_home.shape[0] else 0
+        out = np.zeros((max(nr, 0),) + w_home.shape[1:], dtype=w_home.dtype)
+        self.lib.ora_prefetch_replicas(nr, _p(rep, _i32p), _p(seg, _i32p), row,
+                                       w_home.ctypes.data_as(ctypes.c_void_p),
+                                       out.ctypes.data_as(ctypes.c_void_p))
+        return out
 
 
 _default: Oracle | None = None

@@ -33,7 +33,8 @@
  * of S*K slots; home(e) = e / (E/R); a (rank, expert) segment whose rank is
  * not home(e) is a replica; combine is the K-term weighted sum back to token
  * order; the replica reduction sums an expert's segment rows in ascending
- * segment order.  The backward of dispatch and combine (the training step's
+ * segment order; the replica weight prefetch copies the home expert's weight
+ * row to each replica, in replica-list order.  The backward of dispatch and combine (the training step's
  * return path, [P1-how]: a backward pass exists) is the adjoint of the
  * forward maps: combine's gradient flows to each slot weighted by its router
  * weight, and to each router weight as a dot product with the slot's expert
@@ -347,5 +348,21 @@ void ora_dispatch_backward(int64_t ntok, int K, int64_t H, const int32_t *slot,
             if (absum)
                 absum[g * H + h] = mag;
         }
+    }
+}
+
+/* ---- replica weight prefetch  [P1-how] ---------------------------------- *
+ * The duplicates are given their expert's weights before the expert compute:
+ * w_rep[j, :] = w_home[expert of segment replica_seg[j], :] for every replica
+ * j < num_replicas.  Rows are opaque byte strings of row_bytes (any weight
+ * type).  seg is the plan's {expert, rank, start, count} table. */
+void ora_prefetch_replicas(int32_t num_replicas, const int32_t *replica_seg,
+                           const int32_t *seg, int64_t row_bytes,
+                           const uint8_t *w_home, uint8_t *w_rep)
+{
+    for (int32_t j = 0; j < num_replicas; ++j) {
+        int32_t e = seg[4 * replica_seg[j] + 0];
+        memcpy(w_rep + (int64_t)j * row_bytes, w_home + (int64_t)e * row_bytes,
+               (size_t)row_bytes);
     }
 }

@@ -467,6 +467,29 @@ def pin_dispatch_backward(ora):
     assert np.array_equal(ex, np.repeat((slot + 1).sum(axis=1, keepdims=True).astype(np.float64), H, axis=1))
 
 
+def pin_prefetch_replicas(ora):
+    # brute-force replica list from sorted(); row e of w_home holds e in every byte
+    rng = np.random.default_rng(31)
+    for (R, S, E, K) in [(2, 3, 4, 2), (4, 16, 16, 2), (8, 5, 16, 4), (5, 4, 20, 7)]:
+        idx = _random_idx(rng, R, S, E, K, True, 2.0)
+        pl = ora.plan(R, S, E, K, idx)
+        ref = brute_plan(R, S, E, K, idx)
+        w_home = np.repeat(np.arange(E, dtype=np.uint8)[:, None], 48, axis=1)
+        got = ora.prefetch_replicas(pl, w_home)
+        want = [ref["seg"][s][0] for s in ref["replica_seg"]]
+        assert got.shape[0] == len(want)
+        assert all(np.all(got[j] == want[j]) for j in range(len(want)))
+    # adversarial closed form: replicas are experts 0 (x3) then 1..7 (x4 each)
+    R, S, E, K = 32, 4096, 256, 8
+    idx = np.argsort(-np.random.default_rng(0).standard_normal((R * S, K)), axis=1).astype(np.int32)
+    pl = ora.plan(R, S, E, K, idx)
+    w_home = (np.arange(E, dtype=np.float32)[:, None] + np.arange(4, dtype=np.float32) / 8)
+    got = ora.prefetch_replicas(pl, w_home)
+    experts = [0] * 3 + [e for e in range(1, 8) for _ in range(4)]
+    assert np.array_equal(got, w_home[experts])
+
+
 ALL_PINS = [pin_bf16_widen, pin_bf16_rounding, pin_plan_golden, pin_plan_bruteforce,
             pin_plan_invariants, pin_closed_forms, pin_errors, pin_dispatch,
-            pin_combine, pin_reduce, pin_combine_backward, pin_dispatch_backward]
+            pin_combine, pin_reduce, pin_combine_backward, pin_dispatch_backward,
+            pin_prefetch_replicas]

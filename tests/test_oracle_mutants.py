@@ -65,6 +65,8 @@ MUTANTS = {
     "dispatch_bwd_drops_last_k": (
         "for (int k = 0; k < K; ++k) {\n                double v = (double)ora_bf16_to_f32(grad_buf",
         "for (int k = 0; k < K - 1; ++k) {\n                double v = (double)ora_bf16_to_f32(grad_buf"),
+    "prefetch_uses_rank_not_expert": (
+        "int32_t e = seg[4 * replica_seg[j] + 0];", "int32_t e = seg[4 * replica_seg[j] + 1];"),
 }
 
 
