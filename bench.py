@@ -356,7 +356,8 @@ def main():
                 "frac": kernels[dom]["gbs"] / peak, "traffic": dram_traffic(dom, wl.name),
                 "kernel": dom, "peak_source": f"{peak_kind} hbm_gbs (copy)"}
 
-    # ---- backward of combine and dispatch (timed alone, not part of the step)
+    # ---- backward of combine and dispatch and the replica weight prefetch
+    # (each timed alone, not part of the step)
     backward = None
     if not args.no_backward:
         grad_y = torch.empty_like(buf)
@@ -366,6 +367,11 @@ def main():
                                     N * H * 2 + 2 * NK * H * 2 + NK * 8),
                "dispatch_backward": (lambda: mep.mep_dispatch_backward(s, H, plan, buf, grad_x),
                                      NK * H * 2 + N * H * 2 + NK * 4)}
+        if P:   # replica weight prefetch of expert weights the size of a gradient row
+            nrep = plan.host()["num_replicas"]
+            w_rep = torch.empty_like(G)
+            bwd["prefetch_replica_weights"] = (
+                lambda: mep.mep_prefetch_replica_weights(s, plan, home, w_rep), 2 * nrep * P * 4)
         backward = {}
         for name, (fn, nbytes) in bwd.items():
             ts = []

@@ -178,6 +178,21 @@ MEP_API mep_status_t mep_reduce_replica_grads(mep_shape_t shape, const mep_plan_
                                       int64_t P, const float *seg_grads,
                                       float *home_grads, void *stream);
 
+/* Replica weight prefetch: before the expert compute, every replica gets a
+ * copy of its expert's home weights ("How MoonEP works": the duplicates are
+ * fetched ahead of the main computation).  The forward mirror of
+ * mep_reduce_replica_grads.
+ *   row_bytes  bytes of one expert's weights (any element type), a multiple
+ *              of 16; 0 is a no-op.
+ *   w_home     [E, row_bytes] home weights, 16-byte aligned.
+ *   w_rep      [E+R-1, row_bytes] out: row j < num_replicas receives
+ *              w_home[seg[replica_seg[j]].expert]; rows j >= num_replicas are
+ *              not touched.  num_replicas is read on the device.
+ * Bit-exact copies. */
+MEP_API mep_status_t mep_prefetch_replica_weights(mep_shape_t shape, const mep_plan_t *plan,
+                                                  int64_t row_bytes, const void *w_home,
+                                                  void *w_rep, void *stream);
+
 /* Backward of mep_combine (the adjoint of the weighted combine; the backward
  * pass of "How MoonEP works").
  *   grad_out bf16 [N, H]        gradient of the combine output.

@@ -19,7 +19,7 @@ import torch
 __all__ = [
     "MepError", "Shape", "Plan", "load_library", "library_path",
     "mep_plan_workspace_bytes", "mep_maxvio", "mep_plan", "mep_plan_noalloc", "mep_dispatch",
-    "mep_combine", "mep_combine_backward", "mep_dispatch_backward",
+    "mep_combine", "mep_combine_backward", "mep_dispatch_backward", "mep_prefetch_replica_weights",
     "mep_reduce_replica_grads", "mep_read_status", "mep_status_string",
     "mep_set_wait_limit_ns", "mep_get_wait_limit_ns", "mep_version", "STATUS",
 ]
@@ -34,7 +34,8 @@ STATUS = {0: "MEP_OK", 1: "MEP_ERR_INVALID_ARG", 2: "MEP_ERR_MISALIGNED", 3: "ME
 ABI_SYMBOLS = ("mep_plan_workspace_bytes", "mep_maxvio", "mep_plan", "mep_dispatch", "mep_combine",
                "mep_reduce_replica_grads", "mep_read_status", "mep_status_string",
                "mep_set_wait_limit_ns", "mep_get_wait_limit_ns", "mep_version",
-               "mep_plan_noalloc", "mep_combine_backward", "mep_dispatch_backward")
+               "mep_plan_noalloc", "mep_combine_backward", "mep_dispatch_backward",
+               "mep_prefetch_replica_weights")
 
 
 class MepError(RuntimeError):
@@ -108,6 +109,7 @@ def load_library():
         "mep_plan_noalloc": ([Shape, vp, P, vp], ctypes.c_int),
         "mep_combine_backward": ([Shape, i32, P, vp, vp, vp, vp, vp, vp], ctypes.c_int),
         "mep_dispatch_backward": ([Shape, i32, P, vp, vp, vp], ctypes.c_int),
+        "mep_prefetch_replica_weights": ([Shape, P, i64, vp, vp, vp], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -279,6 +281,21 @@ def mep_dispatch_backward(shape, H: int, plan: Plan, grad_buf, grad_x):
     gx = _need(grad_x, "grad_x", torch.bfloat16, s.N * H, dev)
     _ok(L.mep_dispatch_backward(s, int(H), ctypes.byref(plan.struct), gb, gx, _stream(dev)),
         "mep_dispatch_backward")
+
+
+def mep_prefetch_replica_weights(shape, plan: Plan, w_home, w_rep):
+    """``w_rep[j] = w_home[expert of replica j]`` for j < num_replicas (device
+    count); ``w_home`` ``[E, ...]`` and ``w_rep`` ``[E+R-1, ...]`` of one dtype,
+    rows a multiple of 16 bytes."""
+    L, s = load_library(), _shape(shape)
+    dev = plan.device
+    if w_home.dtype != w_rep.dtype:
+        raise TypeError("w_home and w_rep must have the same dtype")
+    row_bytes = w_home.numel() * w_home.element_size() // max(1, s.E)
+    hp = _need(w_home, "w_home", w_home.dtype, s.E * (row_bytes // w_home.element_size()), dev)
+    rp = _need(w_rep, "w_rep", w_rep.dtype, s.seg_rows * (row_bytes // w_rep.element_size()), dev)
+    _ok(L.mep_prefetch_replica_weights(s, ctypes.byref(plan.struct), int(row_bytes), hp, rp,
+                                       _stream(dev)), "mep_prefetch_replica_weights")
 
 
 def mep_reduce_replica_grads(shape, plan: Plan, P: int, seg_grads, home_grads):

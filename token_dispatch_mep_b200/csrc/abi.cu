@@ -149,6 +149,22 @@ mep_status_t mep_dispatch_backward(mep_shape_t shape, int32_t H, const mep_plan_
   return from_cuda(mep::launch_combine(shape, H, *plan, grad_buf, nullptr, grad_x, as_stream(stream)));
 }
 
+mep_status_t mep_prefetch_replica_weights(mep_shape_t shape, const mep_plan_t *plan,
+                                          int64_t row_bytes, const void *w_home, void *w_rep,
+                                          void *stream) {
+  mep_status_t st = check_shape(shape);
+  if (st != MEP_OK) return st;
+  if (row_bytes < 0 || !plan) return MEP_ERR_INVALID_ARG;
+  if (row_bytes == 0) return MEP_OK;
+  if (!plan->replica_seg || !plan->seg || !plan->num_replicas || !plan->status || !w_home ||
+      !w_rep)
+    return MEP_ERR_INVALID_ARG;
+  if (row_bytes % 16 != 0 || !aligned(w_home, 16) || !aligned(w_rep, 16) ||
+      !aligned(plan->seg, 16) || !aligned(plan->replica_seg, 4) || !aligned(plan->num_replicas, 4))
+    return MEP_ERR_MISALIGNED;
+  return from_cuda(mep::launch_prefetch(shape, *plan, row_bytes, w_home, w_rep, as_stream(stream)));
+}
+
 mep_status_t mep_read_status(const mep_plan_t *plan, void *stream) {
   if (!plan || !plan->status) return MEP_ERR_INVALID_ARG;
   int32_t host = 0;

@@ -32,6 +32,9 @@ cudaError_t launch_combine(const mep_shape_t &s, int32_t H, const mep_plan_t &pl
 cudaError_t launch_reduce(const mep_shape_t &s, const mep_plan_t &pl, int64_t P,
                           const float *G, float *home, cudaStream_t stream);
 
+cudaError_t launch_prefetch(const mep_shape_t &s, const mep_plan_t &pl, int64_t row_bytes,
+                            const void *w_home, void *w_rep, cudaStream_t stream);
+
 cudaError_t launch_combine_backward(const mep_shape_t &s, int32_t H, const mep_plan_t &pl,
                                     const uint16_t *grad_out, const float *w, const uint16_t *y,
                                     uint16_t *grad_y, float *grad_w, cudaStream_t stream);

@@ -1,0 +1,108 @@
+// Replica weight prefetch: w_rep[j, :] = w_home[seg[replica_seg[j]].expert, :]
+// for every replica j < num_replicas; rows are opaque byte strings.
+//
+// Method: the duplicate experts get their weights before the expert compute
+// starts (MoonEP release page, "How MoonEP works"); this is the forward
+// mirror of the replica-gradient reduction.
+//
+// Tasks are (replica, column tile) pairs, replica-major; a tile is kThreads x
+// kU 16-byte vectors.  The number of replicas is read on the device, so the
+// grid has a fixed size and strides over num_replicas x tiles tasks; nothing
+// waits for the host.  Replica indices, segment indices and expert ids are
+// range-checked before any address is formed.  Streaming loads and stores.
+#include <algorithm>
+#include <cstdint>
+
+#include "mep_device.cuh"
+#include "mep_internal.h"
+
+#ifndef MEP_PREFETCH_BLOCKS_PER_SM
+#define MEP_PREFETCH_BLOCKS_PER_SM 32
+#endif
+
+namespace mep {
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kU = 4;
+
+struct PrefetchParams {
+  const uint4 *src;
+  uint4 *dst;
+  const int32_t *replica_seg;
+  const int4 *seg;
+  const int32_t *num_replicas;
+  int32_t *status;
+  int32_t E, rows;  // rows = E + R - 1, the static bound on segments and replicas
+  int64_t cols;     // 16-byte vectors per row
+};
+
+__global__ void __launch_bounds__(kThreads) prefetch_kernel(PrefetchParams p) {
+  int nrep = __ldg(p.num_replicas);
+  bool bad = false;
+  if (nrep < 0 || nrep > p.rows) {
+    bad = true;
+    nrep = 0;
+  }
+  const int64_t tile = (int64_t)kThreads * kU;
+  const int64_t tiles = (p.cols + tile - 1) / tile;
+  const int64_t ntask = (int64_t)nrep * tiles;
+  for (int64_t task = blockIdx.x; task < ntask; task += gridDim.x) {
+    const int j = (int)(task / tiles);
+    const int64_t c0 = (task - (int64_t)j * tiles) * tile + threadIdx.x;
+    const int s = __ldg(p.replica_seg + j);
+    if (s < 0 || s >= p.rows) {
+      bad = true;
+      continue;
+    }
+    const int e = __ldg(&p.seg[s].x);
+    if (e < 0 || e >= p.E) {
+      bad = true;
+      continue;
+    }
+    const uint4 *src = p.src + (int64_t)e * p.cols;
+    uint4 *dst = p.dst + (int64_t)j * p.cols;
+    uint4 v[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int64_t c = c0 + (int64_t)u * kThreads;
+      if (c < p.cols) v[u] = __ldcs(src + c);
+    }
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int64_t c = c0 + (int64_t)u * kThreads;
+      if (c < p.cols) __stcs(dst + c, v[u]);
+    }
+  }
+  if (bad && threadIdx.x == 0) set_status(p.status, MEP_ERR_DEVICE_DATA);
+}
+
+}  // namespace
+
+cudaError_t launch_prefetch(const mep_shape_t &s, const mep_plan_t &pl, int64_t row_bytes,
+                            const void *w_home, void *w_rep, cudaStream_t stream) {
+  int dev = 0, sms = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if ((err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+    return err;
+  PrefetchParams p{};
+  p.src = static_cast<const uint4 *>(w_home);
+  p.dst = static_cast<uint4 *>(w_rep);
+  p.replica_seg = pl.replica_seg;
+  p.seg = reinterpret_cast<const int4 *>(pl.seg);
+  p.num_replicas = pl.num_replicas;
+  p.status = pl.status;
+  p.E = s.E;
+  p.rows = s.E + s.R - 1;
+  p.cols = row_bytes / 16;
+  const int64_t tile = (int64_t)kThreads * kU;
+  const int64_t bound = (int64_t)p.rows * ((p.cols + tile - 1) / tile);
+  const int blocks = (int)std::max<int64_t>(
+      1, std::min<int64_t>(bound, (int64_t)sms * MEP_PREFETCH_BLOCKS_PER_SM));
+  prefetch_kernel<<<blocks, kThreads, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace mep
