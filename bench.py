@@ -9,7 +9,9 @@ mep_dispatch -> mep_combine -> mep_reduce_replica_grads, all through the C ABI.
 
 * value: tokens per second of the whole job (tokens of all ranks / max-over-ranks
   device time), inputs resident in HBM, L2 flushed (512 MB write) between
-  steps outside the timed events.
+  steps outside the timed events.  The step is captured once in a CUDA graph
+  and replayed (``eager`` keeps the launch-by-launch timing, whose per-kernel
+  events give the roofline breakdown).
 * e2e: the same metric through the public API with pinned host buffers: every
   step copies that step's inputs host->device and its outputs (combine
   output, home gradients, plan scalars) back; consecutive steps overlap on
@@ -61,6 +63,8 @@ def parse_args():
                     help="gradient row length (default: the workload's); for small profiling cases")
     ap.add_argument("--e2e-steps", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="skip the CUDA-graph replay timing of the step")
     ap.add_argument("--no-backward", action="store_true",
                     help="skip the separately timed backward kernels")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
@@ -356,6 +360,34 @@ def main():
                 "frac": kernels[dom]["gbs"] / peak, "traffic": dram_traffic(dom, wl.name),
                 "kernel": dom, "peak_source": f"{peak_kind} hbm_gbs (copy)"}
 
+    # ---- the same step captured once in a CUDA graph and replayed
+    graph = None
+    if not args.no_graph:
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(side):
+            step()
+        torch.cuda.current_stream(dev).wait_stream(side)
+        torch.cuda.synchronize()
+        cg = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(cg):
+            step()
+        gts = []
+        for it in range(3 + args.steps):
+            flush.zero_()
+            g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            g0.record()
+            cg.replay()
+            g1.record()
+            if it >= 3:
+                gts.append((g0, g1))
+        torch.cuda.synchronize()
+        gms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in gts])), world, dev)
+        if mep.mep_read_status(plan) != 0:
+            raise RuntimeError("device status not OK after graph replays")
+        graph = {"ms_per_step": gms, "value": whole_job_rate(N, world, gms), "unit": "tokens/s"}
+        del cg
+
     # ---- backward of combine and dispatch and the replica weight prefetch
     # (each timed alone, not part of the step)
     backward = None
@@ -480,6 +512,9 @@ def main():
         cpu = {"value": r["value"], "unit": "tokens/s", "cores": 1, "kind": "oracle",
                "sample": r["sample"], "measured_s": r["measured_s"]}
 
+    eager = {"ms_per_step": ms_step, "value": value, "unit": "tokens/s"}
+    if graph is not None:   # headline: the step as a user runs it, one graph replay per step
+        ms_step, value = graph["ms_per_step"], graph["value"]
     if rank == 0:
         pdc_ms = stage_ms["plan"] + stage_ms["dispatch"] + stage_ms["combine"]
         line = {
@@ -490,6 +525,8 @@ def main():
             "config": {"workload": wl.name, "R": R, "S": S, "E": E, "K": K, "H": H, "P": P,
                        "step": "plan+dispatch+combine+replica-grad reduce",
                        "l2": "flushed by a 512 MB write between steps, outside the events",
+                       "timing": ("CUDA-graph replay of the captured step, events around each replay"
+                                  if graph is not None else "eager launches, events around each kernel"),
                        "parallelism": f"replicas x{world}"},
             "roofline": roofline,
             "cpu_baseline": cpu,
@@ -498,6 +535,8 @@ def main():
             "gpu_launches": launches_per_step * args.steps,
             "stages_ms": stage_ms,
             "backward_kernels": backward,
+            "graph_replay": graph,
+            "eager": eager,
             "kernels": kernels,
             "plan_us": stage_ms["plan"] * 1e3,
             "pdc_tokens_per_s": whole_job_rate(N, world, pdc_ms),
