@@ -88,6 +88,8 @@ class Oracle:
         L.ora_prefetch_replicas.argtypes = [ctypes.c_int32, _i32p, _i32p, ctypes.c_int64,
                                             ctypes.c_void_p, ctypes.c_void_p]
         L.ora_prefetch_replicas.restype = None
+        L.ora_plan_home_first.argtypes = [ctypes.c_int] * 4 + [_i32p] * 12 + [_i32p, _f64p, _i32p]
+        L.ora_plan_home_first.restype = ctypes.c_int
         self.lib = L
 
     # -- scalars -----------------------------------------------------------
@@ -134,6 +136,38 @@ class Oracle:
             out[n] = int(out[n][0])
         out["maxvio"] = float(out["maxvio"][0])
         out["slot"] = out["slot"].reshape(R * S, K)
+        # the contiguous plan lists segments in slot order: each rank's own
+        # segments are the entries rank_seg_ptr[r] .. rank_seg_ptr[r+1]
+        out["rank_seg_idx"] = np.arange(out["num_seg"], dtype=np.int32)
+        return out
+
+    def plan_home_first(self, R, S, E, K, idx) -> dict:
+        """The home-first (low-replica) plan; same fields as ``plan`` plus
+        ``rank_seg_idx``; segments listed by (expert, rank), at most E + R - 1."""
+        idx = np.ascontiguousarray(idx, dtype=np.int32).reshape(-1)
+        NK = R * S * K
+        nseg_max = 2 * E + R
+        out = dict(
+            counts=np.zeros(E, np.int32), expert_offset=np.zeros(E + 1, np.int32),
+            slot=np.zeros(NK, np.int32), src_pair=np.zeros(NK, np.int32),
+            seg=np.zeros((nseg_max, 4), np.int32), num_seg=np.zeros(1, np.int32),
+            num_replicas=np.zeros(1, np.int32), rank_seg_ptr=np.zeros(R + 1, np.int32),
+            rank_seg_idx=np.zeros(nseg_max, np.int32),
+            expert_seg_ptr=np.zeros(E + 1, np.int32), replica_seg=np.zeros(nseg_max, np.int32),
+            max_count=np.zeros(1, np.int32), maxvio=np.zeros(1, np.float64))
+        scratch = np.zeros(6 * E + 3 * R + 2, np.int32)
+        names = ["counts", "expert_offset", "slot", "src_pair", "seg", "num_seg",
+                 "num_replicas", "rank_seg_ptr", "rank_seg_idx", "expert_seg_ptr", "replica_seg",
+                 "max_count"]
+        st = self.lib.ora_plan_home_first(R, S, E, K, _p(idx, _i32p), *[_p(out[n], _i32p) for n in names],
+                                          _p(out["maxvio"], _f64p), _p(scratch, _i32p))
+        if st:
+            raise OracleError(st)
+        for n in ("num_seg", "num_replicas", "max_count"):
+            out[n] = int(out[n][0])
+        out["maxvio"] = float(out["maxvio"][0])
+        out["slot"] = out["slot"].reshape(R * S, K)
+        out["rank_seg_idx"] = out["rank_seg_idx"][:out["num_seg"]].copy()
         return out
 
     # -- data movement ---------------------------------------------------------

@@ -366,3 +366,158 @@ void ora_prefetch_replicas(int32_t num_replicas, const int32_t *replica_seg,
                (size_t)row_bytes);
     }
 }
+
+/* ---- home-first plan (a low-replica schedule; [P1-how] "a small number of
+ * duplicate experts") ------------------------------------------------------ *
+ * Every rank still receives exactly S*K slots.  Reading taken for the pages'
+ * "small number of redundant experts":
+ *   1. each rank fills its S*K slots with its home experts first, in
+ *      ascending expert order: expert e keeps h_e = min(T_e, room left);
+ *   2. the overflow T_e - h_e of every expert, in ascending expert order,
+ *      is cut contiguously over the spare room of the ranks, in ascending
+ *      rank order; each (expert, rank) piece of overflow is a replica;
+ *   3. rank r's slots hold its home pieces (expert order) and then its
+ *      replica pieces (expert order); inside a piece, pairs keep (g, k) order;
+ *      an expert's first h_e pairs are the home ones.
+ * Segments are listed by (expert, rank); rank_seg_idx lists each rank's
+ * segments in slot order (rank r: entries rank_seg_ptr[r] .. rank_seg_ptr[r+1]).
+ * At most E + R - 1 segments: in every full rank at most one expert keeps
+ * only part of its pairs home, so with Z experts keeping none, X overflowing
+ * experts and Y ranks with room there are at most E - Z home pieces and
+ * X + Y - 1 <= (R - Y) + Z + Y - 1 replica pieces.  expert_offset is the exclusive prefix of counts
+ * (the pair's index in the expert-sorted order), not a slot position. */
+int ora_plan_home_first(int R, int S, int E, int K, const int32_t *idx,
+                        int32_t *counts, int32_t *expert_offset, int32_t *slot,
+                        int32_t *src_pair, int32_t *seg, int32_t *num_seg,
+                        int32_t *num_replicas, int32_t *rank_seg_ptr,
+                        int32_t *rank_seg_idx, int32_t *expert_seg_ptr,
+                        int32_t *replica_seg, int32_t *max_count, double *maxvio,
+                        int32_t *scratch /* 6*E + 3*R + 2 ints */)
+{
+    int st = ora_counts(R, S, E, K, idx, counts);
+    if (st)
+        return st;
+    int64_t N = (int64_t)R * S;
+    int64_t C = (int64_t)S * K;
+    int64_t NK = N * K;
+    int B = E / R;
+    *maxvio = ora_maxvio_from_counts(R, S, E, K, counts, max_count);
+    expert_offset[0] = 0;
+    for (int e = 0; e < E; ++e)
+        expert_offset[e + 1] = expert_offset[e] + counts[e];
+
+    int32_t *h = scratch, *pre = h + E, *over = pre + E, *O = over + E;   /* O: E+1 */
+    int32_t *used = O + E + 1;                  /* per-expert pairs placed so far: E */
+    int32_t *F = used + E, *D = F + R;          /* D: R+1 */
+    int32_t *deficit = D + R + 1;               /* R */
+
+    /* 1. home fill, rank by rank, home experts in ascending order */
+    for (int r = 0; r < R; ++r) {
+        int64_t fill = 0;
+        for (int e = r * B; e < (r + 1) * B; ++e) {
+            int64_t take = counts[e] < C - fill ? counts[e] : C - fill;
+            pre[e] = (int32_t)fill;
+            h[e] = (int32_t)take;
+            fill += take;
+        }
+        F[r] = (int32_t)fill;
+        deficit[r] = (int32_t)(C - fill);
+    }
+    /* 2. overflow stream (experts ascending) against spare room (ranks ascending) */
+    O[0] = 0;
+    for (int e = 0; e < E; ++e) {
+        over[e] = counts[e] - h[e];
+        O[e + 1] = O[e] + over[e];
+    }
+    D[0] = 0;
+    for (int r = 0; r < R; ++r)
+        D[r + 1] = D[r] + deficit[r];
+
+    /* 3. place every pair, walking pairs in (g, k) order */
+    for (int e = 0; e < E; ++e)
+        used[e] = 0;
+    for (int64_t pair = 0; pair < NK; ++pair) {      /* pair = g*K + k: (g, k) order */
+        int32_t e = idx[pair];
+        int32_t i = used[e]++;
+        int64_t p;
+        if (i < h[e]) {
+            p = (int64_t)(e / B) * C + pre[e] + i;
+        } else {
+            int64_t q = (int64_t)O[e] + (i - h[e]);
+            int r = 0;
+            while (!(D[r] <= q && q < D[r + 1]))
+                ++r;
+            p = (int64_t)r * C + F[r] + (q - D[r]);
+        }
+        slot[pair] = (int32_t)p;
+        src_pair[p] = (int32_t)pair;
+    }
+
+    /* 4. segments: maximal runs of one expert inside one rank, in slot order,
+     *    then listed by (expert, rank) */
+    int32_t nrun = 0;
+    int32_t prev_r = -1, prev_e = -1;
+    for (int64_t p = 0; p < NK; ++p) {
+        int32_t e = idx[src_pair[p]];
+        int32_t r = (int32_t)(p / C);
+        if (e != prev_e || r != prev_r) {
+            /* temporarily store runs in slot order in seg */
+            seg[4 * nrun + 0] = e;
+            seg[4 * nrun + 1] = r;
+            seg[4 * nrun + 2] = (int32_t)(p - (int64_t)r * C);
+            seg[4 * nrun + 3] = 0;
+            ++nrun;
+            prev_r = r;
+            prev_e = e;
+        }
+        seg[4 * (nrun - 1) + 3] += 1;
+    }
+    *num_seg = nrun;
+    /* stable selection sort of the runs by (expert, rank); rank_seg_idx keeps
+     * each run's new index in slot order */
+    for (int32_t a = 0; a < nrun; ++a)
+        rank_seg_idx[a] = a;                     /* run a (slot order) -> index */
+    for (int32_t a = 0; a < nrun; ++a) {
+        int32_t best = a;
+        for (int32_t b = a + 1; b < nrun; ++b) {
+            int32_t eb = seg[4 * b], rb = seg[4 * b + 1];
+            int32_t ek = seg[4 * best], rk = seg[4 * best + 1];
+            if (eb < ek || (eb == ek && rb < rk))
+                best = b;
+        }
+        if (best != a) {
+            for (int c = 0; c < 4; ++c) {
+                int32_t tmp = seg[4 * a + c];
+                seg[4 * a + c] = seg[4 * best + c];
+                seg[4 * best + c] = tmp;
+            }
+            int32_t tmp = rank_seg_idx[a];
+            rank_seg_idx[a] = rank_seg_idx[best];
+            rank_seg_idx[best] = tmp;
+        }
+    }
+    /* rank_seg_idx[a] now holds the slot-order run id of table entry a;
+     * invert it so that slot-order run j maps to its table index */
+    for (int32_t a = 0; a < nrun; ++a)
+        replica_seg[rank_seg_idx[a]] = a;        /* replica_seg used as scratch */
+    for (int32_t j = 0; j < nrun; ++j)
+        rank_seg_idx[j] = replica_seg[j];
+    int32_t s = 0;
+    for (int r = 0; r <= R; ++r) {               /* runs are rank-major in slot order */
+        while (s < nrun && seg[4 * rank_seg_idx[s] + 1] < r)
+            ++s;
+        rank_seg_ptr[r] = s;
+    }
+    s = 0;
+    for (int e = 0; e <= E; ++e) {
+        while (s < nrun && seg[4 * s] < e)
+            ++s;
+        expert_seg_ptr[e] = s;
+    }
+    int32_t nr = 0;
+    for (int32_t a = 0; a < nrun; ++a)
+        if (seg[4 * a + 1] != seg[4 * a] / B)
+            replica_seg[nr++] = a;
+    *num_replicas = nr;
+    return ORA_OK;
+}

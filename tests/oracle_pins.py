@@ -489,7 +489,137 @@ def pin_prefetch_replicas(ora):
     assert np.array_equal(got, w_home[experts])
 
 
+# ---------------------------------------------------- home-first schedule
+
+def brute_home_first(R, S, E, K, idx):
+    """The home-first plan as a simulation with queues: ranks are bins of
+    S*K slots; each bin takes its home experts' pairs (ascending experts,
+    (g,k) order) while it has room; what does not fit joins one overflow
+    queue; bins are then topped up from the queue in rank order."""
+    idx = np.asarray(idx).reshape(R * S, K)
+    C, B = S * K, E // R
+    lists = [[] for _ in range(E)]
+    for g in range(R * S):
+        for k in range(K):
+            lists[int(idx[g, k])].append(g * K + k)
+    bins = [[] for _ in range(R)]
+    queue = []
+    for r in range(R):
+        for e in range(r * B, (r + 1) * B):
+            room = C - len(bins[r])
+            bins[r] += [(e, q) for q in lists[e][:room]]
+            queue += [(e, q) for q in lists[e][room:]]
+    qi = 0
+    for r in range(R):
+        while len(bins[r]) < C:
+            bins[r].append(queue[qi])
+            qi += 1
+    assert qi == len(queue)
+    slot = np.zeros((R * S, K), np.int64)
+    runs = []                                   # (expert, rank, start, count) in slot order
+    for r in range(R):
+        for i, (e, q) in enumerate(bins[r]):
+            slot[q // K, q % K] = r * C + i
+            if runs and runs[-1][0] == e and runs[-1][1] == r:
+                runs[-1][3] += 1
+            else:
+                runs.append([e, r, i, 1])
+    table = sorted(range(len(runs)), key=lambda j: (runs[j][0], runs[j][1]))
+    where = {j: a for a, j in enumerate(table)}
+    seg = [tuple(runs[j]) for j in table]
+    return dict(slot=slot, seg=seg, rank_seg_idx=[where[j] for j in range(len(runs))],
+                replica_seg=[a for a, sg in enumerate(seg) if sg[1] != sg[0] // B],
+                expert_seg_ptr=[next((a for a, sg in enumerate(seg) if sg[0] >= e), len(seg))
+                                for e in range(E + 1)],
+                rank_seg_ptr=[next((j for j in range(len(runs)) if runs[j][1] >= r), len(runs))
+                              for r in range(R + 1)])
+
+
+def _check_hf_equal(pl, ref, what=""):
+    ns = pl["num_seg"]
+    assert np.array_equal(pl["slot"], ref["slot"]), what
+    assert [tuple(x) for x in pl["seg"][:ns].tolist()] == ref["seg"], what
+    assert list(pl["rank_seg_idx"][:ns]) == ref["rank_seg_idx"], what
+    assert list(pl["rank_seg_ptr"]) == ref["rank_seg_ptr"], what
+    assert list(pl["expert_seg_ptr"]) == ref["expert_seg_ptr"], what
+    assert pl["num_replicas"] == len(ref["replica_seg"]), what
+    assert list(pl["replica_seg"][:pl["num_replicas"]]) == ref["replica_seg"], what
+
+
+def check_home_first_invariants(pl, R, S, E, K, idx):
+    idx = np.asarray(idx).reshape(-1)
+    NK, C, B = R * S * K, S * K, E // R
+    slot = np.asarray(pl["slot"]).reshape(-1).astype(np.int64)
+    src = np.asarray(pl["src_pair"]).astype(np.int64)
+    assert np.array_equal(np.sort(slot), np.arange(NK))           # each pair placed once
+    assert np.array_equal(src[slot], np.arange(NK))
+    ns = pl["num_seg"]
+    seg = np.asarray(pl["seg"])[:ns]
+    assert np.array_equal(np.bincount(seg[:, 1], weights=seg[:, 3], minlength=R), np.full(R, C))
+    e_of_p = idx[src]
+    for e, r, st, cnt in seg:                                       # runs hold one expert
+        assert np.all(e_of_p[r * C + st: r * C + st + cnt] == e)
+    counts = np.bincount(idx, minlength=E)
+    home_load = np.array([counts[r * B:(r + 1) * B].sum() for r in range(R)])
+    over_e = np.zeros(E, np.int64)
+    for e, r, st, cnt in seg:
+        if r != e // B:
+            over_e[e] += cnt
+    for e in range(E):                 # an expert leaves home only if its home rank is full
+        if over_e[e]:
+            assert home_load[e // B] >= C
+    assert ns <= E + R - 1                                          # the static bound
+    deficit_ranks = int((home_load < C).sum())
+    overflowing = int((over_e > 0).sum())
+    if overflowing:
+        assert pl["num_replicas"] <= overflowing + deficit_ranks - 1
+    else:
+        assert pl["num_replicas"] == 0
+
+
+def pin_home_first(ora):
+    gd = load_golden("example_c_home_first.json")
+    pl = ora.plan_home_first(gd["R"], gd["S"], gd["E"], gd["K"], np.array(gd["idx"], np.int32))
+    assert list(pl["counts"]) == gd["counts"] and pl["maxvio"] == gd["maxvio"]
+    assert pl["slot"].tolist() == gd["slot"] and list(pl["src_pair"]) == gd["src_pair"]
+    assert pl["seg"][:pl["num_seg"]].tolist() == gd["segments"]
+    assert list(pl["replica_seg"][:pl["num_replicas"]]) == gd["replica_seg"]
+    assert list(pl["rank_seg_ptr"]) == gd["rank_seg_ptr"]
+    assert list(pl["rank_seg_idx"]) == gd["rank_seg_idx"]
+    assert list(pl["expert_seg_ptr"]) == gd["expert_seg_ptr"]
+    rng = np.random.default_rng(41)
+    for (R, S, E, K) in SMALL_SHAPES:
+        for distinct, skew in ((True, 0.0), (True, 2.5), (False, 0.0)):
+            idx = _random_idx(rng, R, S, E, K, distinct, skew)
+            pl = ora.plan_home_first(R, S, E, K, idx)
+            _check_hf_equal(pl, brute_home_first(R, S, E, K, idx), str((R, S, E, K)))
+            check_home_first_invariants(pl, R, S, E, K, idx)
+    import workloads
+    for name, S in (("kimi_r64_e896_k16", 23), ("skew_r32_zipf1.5", 61), ("r8_e64_h2048", 97)):
+        wl = workloads.reduced(workloads.WORKLOADS[name], S=S)
+        idx, _ = workloads.routing(wl)
+        pl = ora.plan_home_first(wl.R, wl.S, wl.E, wl.K, idx)
+        check_home_first_invariants(pl, wl.R, wl.S, wl.E, wl.K, idx)
+        assert pl["num_replicas"] <= ora.plan(wl.R, wl.S, wl.E, wl.K, idx)["num_replicas"]
+
+
+def pin_home_first_closed_forms(ora):
+    """Where every rank's home experts exactly fill it (round-robin routing)
+    or the overflow order coincides with expert order (adversarial routing),
+    the home-first plan equals the contiguous cut."""
+    import workloads
+    for (R, S, E, K) in [(4, 64, 16, 2), (8, 512, 64, 6), (2, 3, 6, 4)]:
+        idx, _ = workloads.roundrobin_routing(R, S, E, K)
+        a, b = ora.plan_home_first(R, S, E, K, idx), ora.plan(R, S, E, K, idx)
+        assert np.array_equal(a["slot"], b["slot"]) and a["num_replicas"] == 0
+    R, S, E, K = 32, 4096, 256, 8
+    idx = np.argsort(-np.random.default_rng(0).standard_normal((R * S, K)), axis=1).astype(np.int32)
+    a, b = ora.plan_home_first(R, S, E, K, idx), ora.plan(R, S, E, K, idx)
+    assert np.array_equal(a["slot"], b["slot"])
+    assert a["num_seg"] == 32 and a["num_replicas"] == 31
+
+
 ALL_PINS = [pin_bf16_widen, pin_bf16_rounding, pin_plan_golden, pin_plan_bruteforce,
             pin_plan_invariants, pin_closed_forms, pin_errors, pin_dispatch,
             pin_combine, pin_reduce, pin_combine_backward, pin_dispatch_backward,
-            pin_prefetch_replicas]
+            pin_prefetch_replicas, pin_home_first, pin_home_first_closed_forms]

@@ -67,6 +67,12 @@ MUTANTS = {
         "for (int k = 0; k < K - 1; ++k) {\n                double v = (double)ora_bf16_to_f32(grad_buf"),
     "prefetch_uses_rank_not_expert": (
         "int32_t e = seg[4 * replica_seg[j] + 0];", "int32_t e = seg[4 * replica_seg[j] + 1];"),
+    "home_first_fill_ignores_room_order": (
+        "pre[e] = (int32_t)fill;", "pre[e] = (int32_t)(C - fill - take);"),
+    "home_first_overflow_before_home": (
+        "p = (int64_t)r * C + F[r] + (q - D[r]);", "p = (int64_t)r * C + (q - D[r]);"),
+    "home_first_replica_flag_by_slot_rank": (
+        "if (seg[4 * a + 1] != seg[4 * a] / B)", "if (seg[4 * a + 1] != seg[4 * a] % R)"),
 }
 
 
