@@ -360,6 +360,28 @@ def main():
                 "frac": kernels[dom]["gbs"] / peak, "traffic": dram_traffic(dom, wl.name),
                 "kernel": dom, "peak_source": f"{peak_kind} hbm_gbs (copy)"}
 
+    # ---- the home-first (low-replica) plan: latency and replica count
+    home_first = None
+    if not args.no_backward:
+        hf = mep.Plan(s, dev)
+        hts = []
+        for it in range(3 + 20):
+            flush.zero_()
+            h0, h1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            h0.record()
+            mep.mep_plan_home_first(s, idx, hf)
+            h1.record()
+            if it >= 3:
+                hts.append((h0, h1))
+        torch.cuda.synchronize()
+        if mep.mep_read_status(hf) != 0:
+            raise RuntimeError("device status not OK after the home-first plan")
+        hh = hf.host()
+        home_first = {"plan_us": float(np.median([a.elapsed_time(b) for a, b in hts])) * 1e3,
+                      "num_replicas": hh["num_replicas"], "num_seg": hh["num_seg"],
+                      "num_replicas_contiguous": plan.host()["num_replicas"]}
+        del hf
+
     # ---- the same step captured once in a CUDA graph and replayed
     graph = None
     if not args.no_graph:
@@ -536,6 +558,7 @@ def main():
             "stages_ms": stage_ms,
             "backward_kernels": backward,
             "graph_replay": graph,
+            "home_first_plan": home_first,
             "eager": eager,
             "kernels": kernels,
             "plan_us": stage_ms["plan"] * 1e3,

@@ -65,7 +65,7 @@ extern "C" {
 #define MEP_API
 #endif
 
-#define MEP_VERSION 1
+#define MEP_VERSION 2
 #define MEP_MAX_EXPERTS 1024      /* E <= 1024 */
 #define MEP_MAX_RANKS 1024        /* R <= 1024 */
 #define MEP_MAX_HIDDEN 32768      /* H <= 32768 bf16 elements per row */
@@ -95,15 +95,17 @@ typedef struct {
 } mep_segment_t;
 
 /* The plan: device pointers, caller-owned, sized from the shape alone.
- * Segments are ordered by slot, which is also (rank, expert) order and
- * (expert, rank) order; at most E + R - 1 exist. */
+ * Segments are listed by (expert, rank); at most E + R - 1 exist.  In the
+ * contiguous plan (mep_plan) that is also slot order; in the home-first plan
+ * (mep_plan_home_first) each rank's segments in slot order are listed by
+ * rank_seg_idx. */
 typedef struct {
     int32_t *counts;          /* [E]     T_e                                    */
     int32_t *expert_offset;   /* [E+1]   first slot of expert e; [E] = NK        */
     int32_t *slot;            /* [N*K]   pair (g,k) -> global slot p             */
     int32_t *src_pair;        /* [N*K]   slot p -> pair index g*K + k            */
     mep_segment_t *seg;       /* [E+R-1] segments in slot order                  */
-    int32_t *rank_seg_ptr;    /* [R+1]   rank r owns segments [ptr[r], ptr[r+1]) */
+    int32_t *rank_seg_ptr;    /* [R+1]   rank r owns entries [ptr[r], ptr[r+1]) of rank_seg_idx */
     int32_t *expert_seg_ptr;  /* [E+1]   expert e owns segments [ptr[e], ptr[e+1]) */
     int32_t *replica_seg;     /* [E+R-1] indices of replica segments, ascending  */
     int32_t *num_seg;         /* [1]                                             */
@@ -111,6 +113,7 @@ typedef struct {
     int32_t *max_count;       /* [1]     max_e T_e                               */
     int32_t *status;          /* [1]     device error word (mep_status_t)        */
     double *maxvio;           /* [1]     max_e(T_e / T-bar) - 1, T-bar = NK / E  */
+    int32_t *rank_seg_idx;    /* [E+R-1] segment indices, rank by rank, slot order */
 } mep_plan_t;
 
 /* Bytes of workspace mep_plan and mep_maxvio need for this shape.  The
@@ -138,12 +141,35 @@ MEP_API mep_status_t mep_maxvio(mep_shape_t shape, const int32_t *topk_idx,
  *             mep_maxvio; expert_offset = exclusive prefix sum of counts;
  *             slot[g*K+k] = expert_offset[e] + #{(g',k') before (g,k) in
  *             (g, k) order with the same expert e}; src_pair its inverse;
- *             the segments, CSR pointers and replica list of the R-way cut.
+ *             the segments, CSR pointers and replica list of the R-way cut;
+ *             rank_seg_idx[i] = i (segments are already in slot order).
  *             plan->status is cleared at the start of the call.
  * Rank r holds exactly the SK slots [r*SK, (r+1)*SK), in expert order. */
 MEP_API mep_status_t mep_plan(mep_shape_t shape, const int32_t *topk_idx,
                       const mep_plan_t *plan, void *ws, size_t ws_bytes,
                       void *stream);
+
+/* The home-first plan: the same outputs as mep_plan (and the same workspace),
+ * for a schedule that keeps experts home whenever their home rank has room
+ * -- the pages' "small number" of duplicates ("How MoonEP works"); the pages
+ * fix no algorithm, this is the reading this library takes:
+ *   1. rank r fills its S*K slots with its home experts first, in ascending
+ *      expert order: expert e keeps h_e = min(T_e, room left) pairs home;
+ *   2. the overflow T_e - h_e of all experts, in ascending expert order, is
+ *      cut contiguously over the spare room of the ranks in ascending rank
+ *      order; every (expert, rank) piece of overflow is a replica;
+ *   3. rank r's slots hold its home pieces, then its replica pieces, each in
+ *      expert order; inside a piece pairs keep (g, k) order, and an expert's
+ *      first h_e pairs are the ones kept home.
+ * Every rank still receives exactly S*K slots.  Segments are listed by
+ * (expert, rank) (so mep_reduce_replica_grads works unchanged);
+ * rank_seg_idx[rank_seg_ptr[r] .. rank_seg_ptr[r+1]) lists rank r's segments
+ * in slot order.  expert_offset is the exclusive prefix sum of counts (not a
+ * slot position in this plan).  At most E + R - 1 segments, and at most
+ * (overflowing experts) + (ranks with room) - 1 replicas. */
+MEP_API mep_status_t mep_plan_home_first(mep_shape_t shape, const int32_t *topk_idx,
+                                         const mep_plan_t *plan, void *ws, size_t ws_bytes,
+                                         void *stream);
 
 /* Zero-copy dispatch into the static receive buffer ("Why this matters to
  * engineers": each row is copied directly to its final expert-ordered slot).

@@ -82,5 +82,7 @@ def check_plan(gpu: dict, ora: dict, what=""):
     assert np.array_equal(np.asarray(gpu["seg"])[:ns], np.asarray(ora["seg"])[:ns]), f"{what}: seg"
     assert np.array_equal(np.asarray(gpu["replica_seg"])[:nr], np.asarray(ora["replica_seg"])[:nr]), \
         f"{what}: replica_seg"
+    assert np.array_equal(np.asarray(gpu["rank_seg_idx"])[:ns], np.asarray(ora["rank_seg_idx"])[:ns]), \
+        f"{what}: rank_seg_idx"
     assert gpu["maxvio"] == ora["maxvio"], f"{what}: maxvio {gpu['maxvio']!r} vs {ora['maxvio']!r}"
     assert gpu["status"] == 0, f"{what}: status {gpu['status']}"

@@ -43,7 +43,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_version_and_strings(lib):
-    assert mep.mep_version() == 1
+    assert mep.mep_version() == 2
     for code, name in mep.STATUS.items():
         assert mep.mep_status_string(code)
     assert mep.mep_status_string(99) == "unknown status"

@@ -18,7 +18,8 @@ import torch
 
 __all__ = [
     "MepError", "Shape", "Plan", "load_library", "library_path",
-    "mep_plan_workspace_bytes", "mep_maxvio", "mep_plan", "mep_plan_noalloc", "mep_dispatch",
+    "mep_plan_workspace_bytes", "mep_maxvio", "mep_plan", "mep_plan_home_first", "mep_plan_noalloc",
+    "mep_dispatch",
     "mep_combine", "mep_combine_backward", "mep_dispatch_backward", "mep_prefetch_replica_weights",
     "mep_reduce_replica_grads", "mep_read_status", "mep_status_string",
     "mep_set_wait_limit_ns", "mep_get_wait_limit_ns", "mep_version", "STATUS",
@@ -35,7 +36,7 @@ ABI_SYMBOLS = ("mep_plan_workspace_bytes", "mep_maxvio", "mep_plan", "mep_dispat
                "mep_reduce_replica_grads", "mep_read_status", "mep_status_string",
                "mep_set_wait_limit_ns", "mep_get_wait_limit_ns", "mep_version",
                "mep_plan_noalloc", "mep_combine_backward", "mep_dispatch_backward",
-               "mep_prefetch_replica_weights")
+               "mep_prefetch_replica_weights", "mep_plan_home_first")
 
 
 class MepError(RuntimeError):
@@ -72,7 +73,7 @@ class Shape(ctypes.Structure):
 class _PlanStruct(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in (
         "counts", "expert_offset", "slot", "src_pair", "seg", "rank_seg_ptr", "expert_seg_ptr",
-        "replica_seg", "num_seg", "num_replicas", "max_count", "status", "maxvio")]
+        "replica_seg", "num_seg", "num_replicas", "max_count", "status", "maxvio", "rank_seg_idx")]
 
 
 _lib = None
@@ -110,6 +111,7 @@ def load_library():
         "mep_combine_backward": ([Shape, i32, P, vp, vp, vp, vp, vp, vp], ctypes.c_int),
         "mep_dispatch_backward": ([Shape, i32, P, vp, vp, vp], ctypes.c_int),
         "mep_prefetch_replica_weights": ([Shape, P, i64, vp, vp, vp], ctypes.c_int),
+        "mep_plan_home_first": ([Shape, vp, P, vp, sz, vp], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -167,6 +169,7 @@ class Plan:
         self.rank_seg_ptr = torch.zeros(s.R + 1, **i32)
         self.expert_seg_ptr = torch.zeros(s.E + 1, **i32)
         self.replica_seg = torch.zeros(s.seg_rows, **i32)
+        self.rank_seg_idx = torch.zeros(s.seg_rows, **i32)
         self.scalars = torch.zeros(4, **i32)  # num_seg, num_replicas, max_count, status
         self.maxvio_t = torch.zeros(1, dtype=torch.float64, device=self.device)
         nbytes = mep_plan_workspace_bytes(s)
@@ -178,7 +181,7 @@ class Plan:
         self.struct = _PlanStruct(
             a(self.counts), a(self.expert_offset), a(self.slot), a(self.src_pair), a(self.seg),
             a(self.rank_seg_ptr), a(self.expert_seg_ptr), a(self.replica_seg),
-            sc, sc + 4, sc + 8, sc + 12, a(self.maxvio_t))
+            sc, sc + 4, sc + 8, sc + 12, a(self.maxvio_t), a(self.rank_seg_idx))
 
     @property
     def status_tensor(self) -> torch.Tensor:
@@ -196,7 +199,8 @@ class Plan:
             slot=self.slot.cpu().numpy(), src_pair=self.src_pair.cpu().numpy(),
             seg=self.seg.cpu().numpy(), rank_seg_ptr=self.rank_seg_ptr.cpu().numpy(),
             expert_seg_ptr=self.expert_seg_ptr.cpu().numpy(),
-            replica_seg=self.replica_seg.cpu().numpy(), num_seg=sc[0], num_replicas=sc[1],
+            replica_seg=self.replica_seg.cpu().numpy(), rank_seg_idx=self.rank_seg_idx.cpu().numpy(),
+            num_seg=sc[0], num_replicas=sc[1],
             max_count=sc[2], status=sc[3], maxvio=float(self.maxvio_t.item()))
 
 
@@ -227,6 +231,19 @@ def mep_plan(shape, topk_idx, plan: Plan, workspace=None):
     ws_t = plan.workspace if workspace is None else workspace
     ws = _need(ws_t, "workspace", torch.uint8, mep_plan_workspace_bytes(s), dev)
     _ok(L.mep_plan(s, idx, ctypes.byref(plan.struct), ws, ws_t.numel(), _stream(dev)), "mep_plan")
+
+
+def mep_plan_home_first(shape, topk_idx, plan: Plan, workspace=None):
+    """The home-first (low-replica) plan of ``topk_idx`` into ``plan``: every
+    expert stays home while its home rank has room; only overflow becomes
+    replicas.  Same buffers and workspace as ``mep_plan``."""
+    L, s = load_library(), _shape(shape)
+    dev = plan.device
+    idx = _need(topk_idx, "topk_idx", torch.int32, s.NK, dev)
+    ws_t = plan.workspace if workspace is None else workspace
+    ws = _need(ws_t, "workspace", torch.uint8, mep_plan_workspace_bytes(s), dev)
+    _ok(L.mep_plan_home_first(s, idx, ctypes.byref(plan.struct), ws, ws_t.numel(), _stream(dev)),
+        "mep_plan_home_first")
 
 
 def mep_plan_noalloc(shape, topk_idx, plan: Plan):

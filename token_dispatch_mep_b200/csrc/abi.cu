@@ -64,27 +64,42 @@ mep_status_t mep_maxvio(mep_shape_t shape, const int32_t *topk_idx, int32_t *cou
   pl.max_count = max_count;
   pl.maxvio = maxvio;
   pl.status = status;
-  return from_cuda(mep::launch_plan(shape, topk_idx, pl, 0, ws, g_wait_ns.load(), as_stream(stream)));
+  return from_cuda(
+      mep::launch_plan(shape, topk_idx, pl, 0, mep::kPlanContiguous, ws, g_wait_ns.load(), as_stream(stream)));
 }
 
-mep_status_t mep_plan(mep_shape_t shape, const int32_t *topk_idx, const mep_plan_t *plan, void *ws,
-                      size_t ws_bytes, void *stream) {
+namespace {
+
+mep_status_t plan_common(mep_shape_t shape, const int32_t *topk_idx, const mep_plan_t *plan,
+                         void *ws, size_t ws_bytes, void *stream, int kind) {
   mep_status_t st = check_shape(shape);
   if (st != MEP_OK) return st;
   if (!topk_idx || !plan) return MEP_ERR_INVALID_ARG;
   const mep_plan_t &p = *plan;
   if (!p.counts || !p.expert_offset || !p.slot || !p.src_pair || !p.seg || !p.rank_seg_ptr ||
       !p.expert_seg_ptr || !p.replica_seg || !p.num_seg || !p.num_replicas || !p.max_count ||
-      !p.status || !p.maxvio)
+      !p.status || !p.maxvio || !p.rank_seg_idx)
     return MEP_ERR_INVALID_ARG;
   const void *i32s[] = {topk_idx, p.counts, p.expert_offset, p.slot, p.src_pair, p.rank_seg_ptr,
                         p.expert_seg_ptr, p.replica_seg, p.num_seg, p.num_replicas,
-                        p.max_count, p.status};
+                        p.max_count, p.status, p.rank_seg_idx};
   for (const void *q : i32s)
     if (!aligned(q, 4)) return MEP_ERR_MISALIGNED;
   if (!aligned(p.seg, 16) || !aligned(p.maxvio, 8)) return MEP_ERR_MISALIGNED;
   if ((st = check_ws(shape, ws, ws_bytes)) != MEP_OK) return st;
-  return from_cuda(mep::launch_plan(shape, topk_idx, p, 1, ws, g_wait_ns.load(), as_stream(stream)));
+  return from_cuda(mep::launch_plan(shape, topk_idx, p, 1, kind, ws, g_wait_ns.load(), as_stream(stream)));
+}
+
+}  // namespace
+
+mep_status_t mep_plan(mep_shape_t shape, const int32_t *topk_idx, const mep_plan_t *plan, void *ws,
+                      size_t ws_bytes, void *stream) {
+  return plan_common(shape, topk_idx, plan, ws, ws_bytes, stream, mep::kPlanContiguous);
+}
+
+mep_status_t mep_plan_home_first(mep_shape_t shape, const int32_t *topk_idx,
+                                 const mep_plan_t *plan, void *ws, size_t ws_bytes, void *stream) {
+  return plan_common(shape, topk_idx, plan, ws, ws_bytes, stream, mep::kPlanHomeFirst);
 }
 
 mep_status_t mep_dispatch(mep_shape_t shape, int32_t H, const mep_plan_t *plan, const uint16_t *x,

@@ -12,15 +12,18 @@ namespace mep {
 
 constexpr int kPlanThreads = 1024;
 constexpr int kPlanMaxBlocks = 1024;          // bound used to size the workspace
-constexpr int kPlanIdsPerWarp = 512;          // expert ids a plan warp keeps in shared memory
+constexpr int kPlanIdsPerWarp = 448;          // expert ids a plan warp keeps in shared memory
+constexpr int kPlanContiguous = 0;            // plan kinds
+constexpr int kPlanHomeFirst = 1;
 constexpr int64_t kPlanMinPairsPerBlock = 4096;
 constexpr size_t kPlanWsHeader = 256;         // grid-barrier words
 
 size_t plan_workspace_bytes(const mep_shape_t &s);
 
 // full = 1: the whole plan; full = 0: counts, max_count, maxvio, status only.
+// kind: kPlanContiguous (the sorted pairs cut into R chunks) or kPlanHomeFirst.
 cudaError_t launch_plan(const mep_shape_t &s, const int32_t *idx, const mep_plan_t &pl,
-                        int full, void *ws, uint64_t wait_ns, cudaStream_t stream);
+                        int full, int kind, void *ws, uint64_t wait_ns, cudaStream_t stream);
 
 cudaError_t launch_dispatch(const mep_shape_t &s, int32_t H, const mep_plan_t &pl,
                             const uint16_t *x, uint16_t *buf, cudaStream_t stream);

@@ -48,6 +48,7 @@ namespace {
 constexpr int kThreads = kPlanThreads;
 constexpr int kWarps = kThreads / 32;
 constexpr int kBatch = 8;          // 32-pair chunks a warp loads at once
+constexpr int kTab = MEP_MAX_EXPERTS + 1;
 
 #ifndef MEP_PLAN_PEERS_BALLOT
 #define MEP_PLAN_PEERS_BALLOT 1  // 1: peer masks from bit ballots; 0: match.any
@@ -61,9 +62,10 @@ struct PlanParams {
   int32_t nt;    // tiles (nb - 1 with a coordinator, else 1)
   int64_t ppb;   // pairs per tile
   int32_t full;  // 0: counts + maxvio only
+  int32_t kind;  // kPlanContiguous or kPlanHomeFirst
   int32_t *counts, *expert_offset, *slot, *src_pair;
   int4 *seg;
-  int32_t *rank_seg_ptr, *expert_seg_ptr, *replica_seg;
+  int32_t *rank_seg_ptr, *expert_seg_ptr, *replica_seg, *rank_seg_idx;
   int32_t *num_seg, *num_replicas, *max_count, *status;
   double *maxvio;
   int32_t *tile;   // workspace [E][nt]
@@ -127,6 +129,28 @@ __device__ __forceinline__ int block_max(int v, int *s_w) {
   return m;
 }
 
+// First index i in [0, n) with a[i] > x (n if none); a nondecreasing.
+__device__ __forceinline__ int upper_bound_idx(const int *a, int n, int x) {
+  int lo = 0, hi = n;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (a[mid] <= x) lo = mid + 1; else hi = mid;
+  }
+  return lo;
+}
+
+// Slot of the i-th pair (in (g,k) order) of expert e in the home-first plan.
+__device__ __forceinline__ int home_first_slot(int e, int i, int Bx, int C, int R, const int *s_h,
+                                               const int *s_off, const int *s_O, const int *s_F,
+                                               const int *s_D) {
+  const int h = s_h[e];
+  const int home = e / Bx;
+  if (i < h) return home * C + (s_off[e] - s_off[home * Bx]) + i;
+  const int q = s_O[e] + (i - h);
+  const int r = upper_bound_idx(s_D + 1, R, q);  // first rank with D[r+1] > q
+  return r * C + s_F[r] + (q - s_D[r]);
+}
+
 __device__ __forceinline__ bool plan_sync(const PlanParams &p, int k) {
   if (p.nb == 1) {
     __syncthreads();
@@ -138,8 +162,9 @@ __device__ __forceinline__ bool plan_sync(const PlanParams &p, int k) {
 __global__ void __launch_bounds__(kThreads, 1) plan_kernel(PlanParams p) {
   extern __shared__ int smem[];  // [kWarps][E] histograms / cursors, then [kWarps][kPlanIdsPerWarp] ids
   __shared__ int s_w[32];
-  __shared__ int s_off[MEP_MAX_EXPERTS + 1];
-  __shared__ int s_sbase[MEP_MAX_EXPERTS + 1];
+  // Tables over experts (or ranks), E + 1 <= kTab entries each.
+  __shared__ int s_tab[8][kTab];
+  int *s_off = s_tab[0];   // expert offsets (exclusive prefix of T_e), [E] = total
 
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const int E = p.E;
@@ -248,6 +273,9 @@ __global__ void __launch_bounds__(kThreads, 1) plan_kernel(PlanParams p) {
   const int T = t < E ? __ldcg(p.counts + t) : 0;
   int total;
   const int off = block_excl_scan(T, &total, s_w);
+  if (t < E) s_off[t] = off;
+  if (t == 0) s_off[E] = total;
+  __syncthreads();
 
   if (blockIdx.x == 0) {
     const int mx = block_max(T, s_w);
@@ -257,55 +285,174 @@ __global__ void __launch_bounds__(kThreads, 1) plan_kernel(PlanParams p) {
     }
   }
 
-  if (p.full && blockIdx.x == 0) {  // the coordinator (or the only block)
-    const int64_t SK = p.SK;
-    int nseg_e = 0, r0 = 0, r1 = -1;
-    if (t < E && T > 0) {
-      r0 = (int)(off / SK);
-      r1 = (int)((off + (int64_t)T - 1) / SK);
-      nseg_e = r1 - r0 + 1;
-    }
-    int nseg;
-    const int sbase = block_excl_scan(nseg_e, &nseg, s_w);
-    const int home = t / (E / p.R);
-    const int nrep_e = nseg_e - ((nseg_e > 0 && home >= r0 && home <= r1) ? 1 : 0);
-    int nrep;
-    int rbase = block_excl_scan(nrep_e, &nrep, s_w);
+  const int C = (int)p.SK;  // slots per rank
+  const int Bx = E / p.R;   // home experts per rank
+  // Home-first tables, built by every block (they are small): per expert the
+  // pairs kept home h_e and their start pre_e on the home rank, the overflow
+  // prefix O_e and the count of overflowing / home-keeping experts before e;
+  // per rank its home fill F_r and the prefix D_r of the spare room.
+  int *s_h = s_tab[1], *s_O = s_tab[2], *s_F = s_tab[3], *s_D = s_tab[4];
+  int *s_hp = s_tab[5], *s_op = s_tab[6];
+  int h = 0, pre = 0, over = 0;
+  if (p.full && p.kind == kPlanHomeFirst) {
     if (t < E) {
-      s_off[t] = off;
-      s_sbase[t] = sbase;
-      p.expert_offset[t] = off;
-      p.expert_seg_ptr[t] = sbase;
-      for (int j = 0; j < nseg_e; ++j) {
-        const int r = r0 + j;
-        const int64_t lo = max((int64_t)off, (int64_t)r * SK);
-        const int64_t hi = min((int64_t)off + T, (int64_t)(r + 1) * SK);
-        p.seg[sbase + j] = make_int4(t, r, (int)(lo - (int64_t)r * SK), (int)(hi - lo));
-        if (r != home) p.replica_seg[rbase++] = sbase + j;
-      }
+      const int before = off - s_off[(t / Bx) * Bx];  // home experts' pairs before e
+      h = max(0, min(T, C - before));
+      pre = min(before, C);
+      over = T - h;
+    }
+    int otot, hptot, optot;
+    const int O = block_excl_scan(over, &otot, s_w);
+    const int hp = block_excl_scan(h > 0 ? 1 : 0, &hptot, s_w);
+    const int op = block_excl_scan(over > 0 ? 1 : 0, &optot, s_w);
+    int F = 0, room = 0;
+    if (t < p.R) {
+      const int load = s_off[(t + 1) * Bx] - s_off[t * Bx];
+      F = min(load, C);
+      room = C - F;
+    }
+    int dtot;
+    const int D = block_excl_scan(room, &dtot, s_w);
+    if (t < E) {
+      s_h[t] = h;
+      s_O[t] = O;
+      s_hp[t] = hp;
+      s_op[t] = op;
+    }
+    if (t < p.R) {
+      s_F[t] = F;
+      s_D[t] = D;
     }
     if (t == 0) {
-      s_off[E] = total;
-      s_sbase[E] = nseg;
-      p.expert_offset[E] = total;
-      p.expert_seg_ptr[E] = nseg;
-      *p.num_seg = nseg;
-      *p.num_replicas = nrep;
+      s_O[E] = otot;
+      s_hp[E] = hptot;
+      s_op[E] = optot;
+      s_D[p.R] = dtot;
     }
     __syncthreads();
-    for (int r = t; r <= p.R; r += kThreads) {
-      const int64_t x = (int64_t)r * SK;
-      int ptr = nseg;
-      if (r < p.R && x < total) {
-        int lo = 0, hi = E + 1;  // first index with s_off > x
-        while (lo < hi) {
-          const int mid = (lo + hi) >> 1;
-          if ((int64_t)s_off[mid] <= x) lo = mid + 1; else hi = mid;
-        }
-        const int e = lo - 1;
-        ptr = s_sbase[e] + (r - (int)(s_off[e] / SK));
+  }
+
+  if (p.full && blockIdx.x == 0) {  // the coordinator (or the only block)
+    if (p.kind == kPlanContiguous) {
+      const int64_t SK = p.SK;
+      int *s_sbase = s_tab[1];
+      int nseg_e = 0, r0 = 0, r1 = -1;
+      if (t < E && T > 0) {
+        r0 = (int)(off / SK);
+        r1 = (int)((off + (int64_t)T - 1) / SK);
+        nseg_e = r1 - r0 + 1;
       }
-      p.rank_seg_ptr[r] = ptr;
+      int nseg;
+      const int sbase = block_excl_scan(nseg_e, &nseg, s_w);
+      const int home = t / Bx;
+      const int nrep_e = nseg_e - ((nseg_e > 0 && home >= r0 && home <= r1) ? 1 : 0);
+      int nrep;
+      int rbase = block_excl_scan(nrep_e, &nrep, s_w);
+      if (t < E) {
+        s_sbase[t] = sbase;
+        p.expert_offset[t] = off;
+        p.expert_seg_ptr[t] = sbase;
+        for (int j = 0; j < nseg_e; ++j) {
+          const int r = r0 + j;
+          const int64_t lo = max((int64_t)off, (int64_t)r * SK);
+          const int64_t hi = min((int64_t)off + T, (int64_t)(r + 1) * SK);
+          p.seg[sbase + j] = make_int4(t, r, (int)(lo - (int64_t)r * SK), (int)(hi - lo));
+          p.rank_seg_idx[sbase + j] = sbase + j;  // slot order is table order
+          if (r != home) p.replica_seg[rbase++] = sbase + j;
+        }
+      }
+      if (t == 0) {
+        s_sbase[E] = nseg;
+        p.expert_offset[E] = total;
+        p.expert_seg_ptr[E] = nseg;
+        *p.num_seg = nseg;
+        *p.num_replicas = nrep;
+      }
+      __syncthreads();
+      for (int r = t; r <= p.R; r += kThreads) {
+        const int64_t x = (int64_t)r * SK;
+        int ptr = nseg;
+        if (r < p.R && x < total) {
+          int lo = 0, hi = E + 1;  // first index with s_off > x
+          while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if ((int64_t)s_off[mid] <= x) lo = mid + 1; else hi = mid;
+          }
+          const int e = lo - 1;
+          ptr = s_sbase[e] + (r - (int)(s_off[e] / SK));
+        }
+        p.rank_seg_ptr[r] = ptr;
+      }
+    } else {
+      int *s_rsp = s_tab[7];
+      const int R = p.R;
+      // Per rank: home pieces (home experts keeping pairs) + replica pieces
+      // (overflowing experts whose overflow meets the rank's spare room).
+      int nh = 0, nr = 0;
+      if (t < R) {
+        nh = s_hp[(t + 1) * Bx] - s_hp[t * Bx];
+        const int d0 = s_D[t], d1 = s_D[t + 1];
+        if (d1 > d0) {
+          const int ef = upper_bound_idx(s_O, E + 1, d0) - 1;       // expert holding d0
+          const int el = upper_bound_idx(s_O, E + 1, d1 - 1) - 1;   // expert holding d1 - 1
+          nr = s_op[el + 1] - s_op[ef];
+        }
+      }
+      int ntot;
+      const int rsp = block_excl_scan(nh + nr, &ntot, s_w);
+      if (t < R) {
+        s_rsp[t] = rsp;
+        p.rank_seg_ptr[t] = rsp;
+      }
+      if (t == 0) {
+        s_rsp[R] = ntot;
+        p.rank_seg_ptr[R] = ntot;
+      }
+      __syncthreads();
+      // Per expert: its pieces in rank order (the home piece sits among the
+      // replica pieces by rank).
+      int rf = 0, rl = -1;
+      if (t < E && over > 0) {
+        const int O = s_O[t];
+        rf = upper_bound_idx(s_D + 1, R, O);                 // first rank with D[r+1] > O
+        rl = upper_bound_idx(s_D + 1, R, O + over - 1);      // rank holding the last pair
+      }
+      int nrep_e = 0;
+      for (int r = rf; r <= rl; ++r)
+        if (s_D[r + 1] > s_D[r]) ++nrep_e;
+      const int nseg_e = nrep_e + (h > 0 ? 1 : 0);
+      int nseg, nrep;
+      int sidx = block_excl_scan(nseg_e, &nseg, s_w);
+      int ridx = block_excl_scan(nrep_e, &nrep, s_w);
+      if (t < E) {
+        const int home = t / Bx;
+        p.expert_offset[t] = off;
+        p.expert_seg_ptr[t] = sidx;
+        const int O = s_O[t];
+        bool home_done = h == 0;
+        for (int r = rf; r <= rl + 1; ++r) {
+          if (!home_done && (r > rl || r > home)) {  // home piece, in rank order
+            p.seg[sidx] = make_int4(t, home, pre, h);
+            p.rank_seg_idx[s_rsp[home] + (s_hp[t] - s_hp[home * Bx])] = sidx;
+            ++sidx;
+            home_done = true;
+          }
+          if (r > rl || s_D[r + 1] <= s_D[r]) continue;
+          const int lo = max(O, s_D[r]), hi = min(O + over, s_D[r + 1]);
+          p.seg[sidx] = make_int4(t, r, s_F[r] + (lo - s_D[r]), hi - lo);
+          const int ef = upper_bound_idx(s_O, E + 1, s_D[r]) - 1;
+          const int nh_r = s_hp[(r + 1) * Bx] - s_hp[r * Bx];
+          p.rank_seg_idx[s_rsp[r] + nh_r + (s_op[t] - s_op[ef])] = sidx;
+          p.replica_seg[ridx++] = sidx;
+          ++sidx;
+        }
+      }
+      if (t == 0) {
+        p.expert_offset[E] = total;
+        p.expert_seg_ptr[E] = nseg;
+        *p.num_seg = nseg;
+        *p.num_replicas = nrep;
+      }
     }
   }
 
@@ -317,6 +464,7 @@ __global__ void __launch_bounds__(kThreads, 1) plan_kernel(PlanParams p) {
     }
     __syncthreads();
 
+    const bool hf = p.kind == kPlanHomeFirst;
     const unsigned lt = lanemask_lt();
     for (int64_t c = w0; c < w1; c += 32) {
       const int64_t q = c + lane;
@@ -328,7 +476,8 @@ __global__ void __launch_bounds__(kThreads, 1) plan_kernel(PlanParams p) {
       const int base = valid ? wh[e] : 0;
       __syncwarp();
       if (valid) {
-        const int s = base + __popc(peers & lt);
+        int s = base + __popc(peers & lt);  // position in the expert-sorted order
+        if (hf) s = home_first_slot(e, s - s_off[e], Bx, C, p.R, s_h, s_off, s_O, s_F, s_D);
         p.slot[q] = s;
         if ((unsigned)s < (unsigned)p.NK) p.src_pair[s] = (int32_t)q;
         if (lane == __ffs(peers) - 1) wh[e] = base + __popc(peers);
@@ -356,7 +505,7 @@ size_t plan_workspace_bytes(const mep_shape_t &s) {
 }
 
 cudaError_t launch_plan(const mep_shape_t &s, const int32_t *idx, const mep_plan_t &pl,
-                        int full, void *ws, uint64_t wait_ns, cudaStream_t stream) {
+                        int full, int kind, void *ws, uint64_t wait_ns, cudaStream_t stream) {
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
@@ -390,6 +539,8 @@ cudaError_t launch_plan(const mep_shape_t &s, const int32_t *idx, const mep_plan
   p.nt = nt;
   p.ppb = (NK + nt - 1) / nt;
   p.full = full;
+  p.kind = kind;
+  p.rank_seg_idx = pl.rank_seg_idx;
   p.counts = pl.counts; p.expert_offset = pl.expert_offset; p.slot = pl.slot;
   p.src_pair = pl.src_pair; p.seg = reinterpret_cast<int4 *>(pl.seg);
   p.rank_seg_ptr = pl.rank_seg_ptr; p.expert_seg_ptr = pl.expert_seg_ptr;
