@@ -204,6 +204,26 @@ MEP_API mep_status_t mep_reduce_replica_grads(mep_shape_t shape, const mep_plan_
                                       int64_t P, const float *seg_grads,
                                       float *home_grads, void *stream);
 
+/* Rank-addressed dispatch and combine: the same operations with every rank's
+ * S*K slots in a buffer of its own.  This is the form the exchange between
+ * GPUs takes: on a multi-GPU system rank r's receive buffer lives on GPU r
+ * and is mapped into this GPU's address space (CUDA IPC or symmetric memory
+ * over NVLink), so each 16-byte store of dispatch is a peer write straight
+ * into the slot that rank owns and combine reads its rows back the same way
+ * -- the all-to-all is fused into the copy, with no staging buffer.  The
+ * caller orders the exchange (every rank's buffer free before dispatch, every
+ * rank's expert outputs written before combine).
+ *   rank_bufs / rank_ys  device array of R device pointers (8-byte aligned);
+ *            pointer r addresses rank r's [S*K, H] bf16 rows, 16-byte aligned.
+ *   Slot p is row p % (S*K) of buffer p / (S*K).  Results are bit-identical
+ *   to mep_dispatch / mep_combine on the concatenated buffer. */
+MEP_API mep_status_t mep_dispatch_ranked(mep_shape_t shape, int32_t H, const mep_plan_t *plan,
+                                         const uint16_t *x, uint16_t *const *rank_bufs,
+                                         void *stream);
+MEP_API mep_status_t mep_combine_ranked(mep_shape_t shape, int32_t H, const mep_plan_t *plan,
+                                        const uint16_t *const *rank_ys, const float *topk_w,
+                                        uint16_t *out, void *stream);
+
 /* Replica weight prefetch: before the expert compute, every replica gets a
  * copy of its expert's home weights ("How MoonEP works": the duplicates are
  * fetched ahead of the main computation).  The forward mirror of

@@ -21,6 +21,7 @@ __all__ = [
     "mep_plan_workspace_bytes", "mep_maxvio", "mep_plan", "mep_plan_home_first", "mep_plan_noalloc",
     "mep_dispatch",
     "mep_combine", "mep_combine_backward", "mep_dispatch_backward", "mep_prefetch_replica_weights",
+    "mep_dispatch_ranked", "mep_combine_ranked", "rank_pointer_table",
     "mep_reduce_replica_grads", "mep_read_status", "mep_status_string",
     "mep_set_wait_limit_ns", "mep_get_wait_limit_ns", "mep_version", "STATUS",
 ]
@@ -36,7 +37,8 @@ ABI_SYMBOLS = ("mep_plan_workspace_bytes", "mep_maxvio", "mep_plan", "mep_dispat
                "mep_reduce_replica_grads", "mep_read_status", "mep_status_string",
                "mep_set_wait_limit_ns", "mep_get_wait_limit_ns", "mep_version",
                "mep_plan_noalloc", "mep_combine_backward", "mep_dispatch_backward",
-               "mep_prefetch_replica_weights", "mep_plan_home_first")
+               "mep_prefetch_replica_weights", "mep_plan_home_first", "mep_dispatch_ranked",
+               "mep_combine_ranked")
 
 
 class MepError(RuntimeError):
@@ -112,6 +114,8 @@ def load_library():
         "mep_dispatch_backward": ([Shape, i32, P, vp, vp, vp], ctypes.c_int),
         "mep_prefetch_replica_weights": ([Shape, P, i64, vp, vp, vp], ctypes.c_int),
         "mep_plan_home_first": ([Shape, vp, P, vp, sz, vp], ctypes.c_int),
+        "mep_dispatch_ranked": ([Shape, i32, P, vp, vp, vp], ctypes.c_int),
+        "mep_combine_ranked": ([Shape, i32, P, vp, vp, vp, vp], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -313,6 +317,38 @@ def mep_prefetch_replica_weights(shape, plan: Plan, w_home, w_rep):
     rp = _need(w_rep, "w_rep", w_rep.dtype, s.seg_rows * (row_bytes // w_rep.element_size()), dev)
     _ok(L.mep_prefetch_replica_weights(s, ctypes.byref(plan.struct), int(row_bytes), hp, rp,
                                        _stream(dev)), "mep_prefetch_replica_weights")
+
+
+def rank_pointer_table(bufs, shape, H: int, device) -> torch.Tensor:
+    """Device array of the R rank buffers' addresses (each [S*K, H] bf16)."""
+    s = _shape(shape)
+    if len(bufs) != s.R:
+        raise ValueError(f"{len(bufs)} rank buffers, need {s.R}")
+    for r, b in enumerate(bufs):
+        _need(b, f"rank buffer {r}", torch.bfloat16, s.SK * H, torch.device(device))
+    return torch.tensor([b.data_ptr() for b in bufs], dtype=torch.int64, device=device)
+
+
+def mep_dispatch_ranked(shape, H: int, plan: Plan, x, rank_table):
+    """Dispatch into R separate rank buffers; ``rank_table`` from
+    ``rank_pointer_table`` (keep the buffers alive while it is used)."""
+    L, s = load_library(), _shape(shape)
+    dev = plan.device
+    xp = _need(x, "x", torch.bfloat16, s.N * H, dev)
+    tp = _need(rank_table, "rank_table", torch.int64, s.R, dev)
+    _ok(L.mep_dispatch_ranked(s, int(H), ctypes.byref(plan.struct), xp, tp, _stream(dev)),
+        "mep_dispatch_ranked")
+
+
+def mep_combine_ranked(shape, H: int, plan: Plan, rank_table, topk_w, out):
+    """Combine reading expert outputs from R separate rank buffers."""
+    L, s = load_library(), _shape(shape)
+    dev = plan.device
+    tp = _need(rank_table, "rank_table", torch.int64, s.R, dev)
+    wp = _need(topk_w, "topk_w", torch.float32, s.NK, dev)
+    op = _need(out, "out", torch.bfloat16, s.N * H, dev)
+    _ok(L.mep_combine_ranked(s, int(H), ctypes.byref(plan.struct), tp, wp, op, _stream(dev)),
+        "mep_combine_ranked")
 
 
 def mep_reduce_replica_grads(shape, plan: Plan, P: int, seg_grads, home_grads):

@@ -109,7 +109,7 @@ mep_status_t mep_dispatch(mep_shape_t shape, int32_t H, const mep_plan_t *plan, 
   if ((st = check_hidden(H)) != MEP_OK) return st;
   if (!plan || !plan->slot || !plan->status || !x || !buf) return MEP_ERR_INVALID_ARG;
   if (!aligned(x, 16) || !aligned(buf, 16) || !aligned(plan->slot, 4)) return MEP_ERR_MISALIGNED;
-  return from_cuda(mep::launch_dispatch(shape, H, *plan, x, buf, as_stream(stream)));
+  return from_cuda(mep::launch_dispatch(shape, H, *plan, x, buf, nullptr, as_stream(stream)));
 }
 
 mep_status_t mep_combine(mep_shape_t shape, int32_t H, const mep_plan_t *plan, const uint16_t *y,
@@ -120,7 +120,7 @@ mep_status_t mep_combine(mep_shape_t shape, int32_t H, const mep_plan_t *plan, c
   if (!plan || !plan->slot || !plan->status || !y || !topk_w || !out) return MEP_ERR_INVALID_ARG;
   if (!aligned(y, 16) || !aligned(out, 16) || !aligned(topk_w, 4) || !aligned(plan->slot, 4))
     return MEP_ERR_MISALIGNED;
-  return from_cuda(mep::launch_combine(shape, H, *plan, y, topk_w, out, as_stream(stream)));
+  return from_cuda(mep::launch_combine(shape, H, *plan, y, nullptr, topk_w, out, as_stream(stream)));
 }
 
 mep_status_t mep_reduce_replica_grads(mep_shape_t shape, const mep_plan_t *plan, int64_t P,
@@ -161,7 +161,8 @@ mep_status_t mep_dispatch_backward(mep_shape_t shape, int32_t H, const mep_plan_
   if (!plan || !plan->slot || !plan->status || !grad_buf || !grad_x) return MEP_ERR_INVALID_ARG;
   if (!aligned(grad_buf, 16) || !aligned(grad_x, 16) || !aligned(plan->slot, 4))
     return MEP_ERR_MISALIGNED;
-  return from_cuda(mep::launch_combine(shape, H, *plan, grad_buf, nullptr, grad_x, as_stream(stream)));
+  return from_cuda(
+      mep::launch_combine(shape, H, *plan, grad_buf, nullptr, nullptr, grad_x, as_stream(stream)));
 }
 
 mep_status_t mep_prefetch_replica_weights(mep_shape_t shape, const mep_plan_t *plan,
@@ -178,6 +179,29 @@ mep_status_t mep_prefetch_replica_weights(mep_shape_t shape, const mep_plan_t *p
       !aligned(plan->seg, 16) || !aligned(plan->replica_seg, 4) || !aligned(plan->num_replicas, 4))
     return MEP_ERR_MISALIGNED;
   return from_cuda(mep::launch_prefetch(shape, *plan, row_bytes, w_home, w_rep, as_stream(stream)));
+}
+
+mep_status_t mep_dispatch_ranked(mep_shape_t shape, int32_t H, const mep_plan_t *plan,
+                                 const uint16_t *x, uint16_t *const *rank_bufs, void *stream) {
+  mep_status_t st = check_shape(shape);
+  if (st != MEP_OK) return st;
+  if ((st = check_hidden(H)) != MEP_OK) return st;
+  if (!plan || !plan->slot || !plan->status || !x || !rank_bufs) return MEP_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(rank_bufs, 8) || !aligned(plan->slot, 4)) return MEP_ERR_MISALIGNED;
+  return from_cuda(mep::launch_dispatch(shape, H, *plan, x, nullptr, rank_bufs, as_stream(stream)));
+}
+
+mep_status_t mep_combine_ranked(mep_shape_t shape, int32_t H, const mep_plan_t *plan,
+                                const uint16_t *const *rank_ys, const float *topk_w, uint16_t *out,
+                                void *stream) {
+  mep_status_t st = check_shape(shape);
+  if (st != MEP_OK) return st;
+  if ((st = check_hidden(H)) != MEP_OK) return st;
+  if (!plan || !plan->slot || !plan->status || !rank_ys || !topk_w || !out)
+    return MEP_ERR_INVALID_ARG;
+  if (!aligned(rank_ys, 8) || !aligned(out, 16) || !aligned(topk_w, 4) || !aligned(plan->slot, 4))
+    return MEP_ERR_MISALIGNED;
+  return from_cuda(mep::launch_combine(shape, H, *plan, nullptr, rank_ys, topk_w, out, as_stream(stream)));
 }
 
 mep_status_t mep_read_status(const mep_plan_t *plan, void *stream) {

@@ -15,6 +15,9 @@
 // loads before it touches any of them, adds them in k order with float32
 // FMAs, rounds to bf16 and writes 16 bytes per chunk (streaming store).
 //
+// Rank-addressed form (mep_combine_ranked): expert outputs are read from R
+// separate rank buffers, slot p being row p % SK of rank_ys[p / SK].
+//
 // With no weights (w == nullptr) every weight is 1 and the kernel is the
 // backward of dispatch: grad_x[g] = bf16(sum_k grad_buf[slot[g,k]]) (an FMA
 // with weight 1 rounds exactly like an addition).
@@ -48,6 +51,8 @@ constexpr int kWarps = kThreads / 32;
 
 struct CombineParams {
   const uint16_t *y;
+  const uint16_t *const *rank_ys;  // ranked form: R row buffers of SK rows
+  int64_t SK;
   const float *w;
   const int32_t *slot;
   uint16_t *out;
@@ -79,7 +84,7 @@ __device__ __forceinline__ uint4 pack8(const float (&acc)[8]) {
   return make_uint4(u[0], u[1], u[2], u[3]);
 }
 
-template <int KC, int U>
+template <int KC, int U, bool kRanked>
 __global__ void __launch_bounds__(kThreads, MEP_COMBINE_MIN_BLOCKS) combine_kernel(CombineParams p) {
   const int lane = threadIdx.x & 31;
   const int64_t nwarps = (int64_t)gridDim.x * kWarps;
@@ -112,7 +117,15 @@ __global__ void __launch_bounds__(kThreads, MEP_COMBINE_MIN_BLOCKS) combine_kern
       if (k < p.K) {
         const bool ok = (unsigned)pk < (unsigned)p.NK;
         bad |= !ok;
-        const uint4 *row = reinterpret_cast<const uint4 *>(p.y + (int64_t)(ok ? pk : 0) * p.H);
+        const int64_t pp = ok ? pk : 0;
+        const uint16_t *yrow;
+        if (kRanked) {
+          const int64_t r = pp / p.SK;
+          yrow = p.rank_ys[r] + (pp - r * p.SK) * p.H;
+        } else {
+          yrow = p.y + pp * p.H;
+        }
+        const uint4 *row = reinterpret_cast<const uint4 *>(yrow);
 #pragma unroll
         for (int u = 0; u < U; ++u) {
           const int c = cbase + u * 32;
@@ -154,15 +167,18 @@ cudaError_t launch_kc(CombineParams p, int sms, cudaStream_t stream) {
   const int64_t want = (ntask + kWarps - 1) / kWarps;
   const int blocks = (int)std::max<int64_t>(
       1, std::min<int64_t>(want, (int64_t)sms * MEP_COMBINE_BLOCKS_PER_SM));
-  combine_kernel<KC, U><<<blocks, kThreads, 0, stream>>>(p);
+  if (p.rank_ys != nullptr)
+    combine_kernel<KC, U, true><<<blocks, kThreads, 0, stream>>>(p);
+  else
+    combine_kernel<KC, U, false><<<blocks, kThreads, 0, stream>>>(p);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_combine(const mep_shape_t &s, int32_t H, const mep_plan_t &pl,
-                           const uint16_t *y, const float *w, uint16_t *out,
-                           cudaStream_t stream) {
+                           const uint16_t *y, const uint16_t *const *rank_ys, const float *w,
+                           uint16_t *out, cudaStream_t stream) {
   int dev = 0, sms = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
@@ -170,6 +186,8 @@ cudaError_t launch_combine(const mep_shape_t &s, int32_t H, const mep_plan_t &pl
     return err;
   CombineParams p{};
   p.y = y;
+  p.rank_ys = rank_ys;
+  p.SK = (int64_t)s.S * s.K;
   p.w = w;
   p.slot = pl.slot;
   p.out = out;

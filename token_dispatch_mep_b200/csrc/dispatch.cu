@@ -17,6 +17,11 @@
 // (uneven destination rows balance out).  Every slot is bounds-checked
 // against [0, N*K) before it is used.
 //
+// Rank-addressed form (mep_dispatch_ranked): rank r's S*K slots live in
+// their own buffer rank_bufs[r] (on a multi-GPU system a peer buffer mapped
+// into this GPU's address space), so slot p is row p % SK of rank_bufs[p / SK]
+// and each store goes straight to the rank that owns the slot.
+//
 // A bulk-copy (TMA) design -- rows staged in shared memory by bulk loads on
 // mbarriers, K bulk stores per row -- measured 0.82-0.87 of the HBM copy
 // peak on this path against 0.89-0.94 for this one, so it is not used.
@@ -44,6 +49,8 @@ constexpr int kU = MEP_DISPATCH_U;
 struct DispatchParams {
   const uint16_t *x;
   uint16_t *buf;
+  uint16_t *const *rank_bufs;  // ranked form: R row buffers of SK rows
+  int64_t SK;
   const int32_t *slot;
   int32_t *status;
   int64_t N, NK;
@@ -52,7 +59,7 @@ struct DispatchParams {
   int32_t parts;   // warp tasks per token
 };
 
-template <int KC>
+template <int KC, bool kRanked>
 __global__ void __launch_bounds__(kThreads) dispatch_kernel(DispatchParams p) {
   const int lane = threadIdx.x & 31;
   const int64_t nwarps = (int64_t)gridDim.x * kWarps;
@@ -79,7 +86,14 @@ __global__ void __launch_bounds__(kThreads) dispatch_kernel(DispatchParams p) {
       const int pk = __shfl_sync(0xffffffffu, sl, k);
       if (k < p.K) {
         if ((unsigned)pk < (unsigned)p.NK) {
-          uint4 *brow = reinterpret_cast<uint4 *>(p.buf + (int64_t)pk * p.H);
+          uint16_t *row;
+          if (kRanked) {
+            const int64_t r = pk / p.SK;
+            row = p.rank_bufs[r] + (pk - r * p.SK) * p.H;
+          } else {
+            row = p.buf + (int64_t)pk * p.H;
+          }
+          uint4 *brow = reinterpret_cast<uint4 *>(row);
 #pragma unroll
           for (int u = 0; u < kU; ++u) {
             const int c = cbase + u * 32;
@@ -100,14 +114,18 @@ cudaError_t launch_kc(const DispatchParams &p, int sms, cudaStream_t stream) {
   const int64_t want = (p.N * p.parts + kWarps - 1) / kWarps;
   const int blocks = (int)std::max<int64_t>(
       1, std::min<int64_t>(want, (int64_t)sms * MEP_DISPATCH_BLOCKS_PER_SM));
-  dispatch_kernel<KC><<<blocks, kThreads, 0, stream>>>(p);
+  if (p.rank_bufs != nullptr)
+    dispatch_kernel<KC, true><<<blocks, kThreads, 0, stream>>>(p);
+  else
+    dispatch_kernel<KC, false><<<blocks, kThreads, 0, stream>>>(p);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_dispatch(const mep_shape_t &s, int32_t H, const mep_plan_t &pl,
-                            const uint16_t *x, uint16_t *buf, cudaStream_t stream) {
+                            const uint16_t *x, uint16_t *buf, uint16_t *const *rank_bufs,
+                            cudaStream_t stream) {
   int dev = 0, sms = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
@@ -116,6 +134,8 @@ cudaError_t launch_dispatch(const mep_shape_t &s, int32_t H, const mep_plan_t &p
   DispatchParams p{};
   p.x = x;
   p.buf = buf;
+  p.rank_bufs = rank_bufs;
+  p.SK = (int64_t)s.S * s.K;
   p.slot = pl.slot;
   p.status = pl.status;
   p.N = (int64_t)s.R * s.S;

@@ -25,12 +25,15 @@ size_t plan_workspace_bytes(const mep_shape_t &s);
 cudaError_t launch_plan(const mep_shape_t &s, const int32_t *idx, const mep_plan_t &pl,
                         int full, int kind, void *ws, uint64_t wait_ns, cudaStream_t stream);
 
+// rank_bufs / rank_ys: nullptr for one [R, S*K, H] buffer, else a device array
+// of R row buffers of S*K rows each.
 cudaError_t launch_dispatch(const mep_shape_t &s, int32_t H, const mep_plan_t &pl,
-                            const uint16_t *x, uint16_t *buf, cudaStream_t stream);
+                            const uint16_t *x, uint16_t *buf, uint16_t *const *rank_bufs,
+                            cudaStream_t stream);
 
 cudaError_t launch_combine(const mep_shape_t &s, int32_t H, const mep_plan_t &pl,
-                           const uint16_t *y, const float *w, uint16_t *out,
-                           cudaStream_t stream);
+                           const uint16_t *y, const uint16_t *const *rank_ys, const float *w,
+                           uint16_t *out, cudaStream_t stream);
 
 cudaError_t launch_reduce(const mep_shape_t &s, const mep_plan_t &pl, int64_t P,
                           const float *G, float *home, cudaStream_t stream);
