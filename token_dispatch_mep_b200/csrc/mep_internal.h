@@ -15,7 +15,10 @@ constexpr int kPlanMaxBlocks = 1024;          // bound used to size the workspac
 constexpr int kPlanIdsPerWarp = 448;          // expert ids a plan warp keeps in shared memory
 constexpr int kPlanContiguous = 0;            // plan kinds
 constexpr int kPlanHomeFirst = 1;
-constexpr int64_t kPlanMinPairsPerBlock = 4096;
+#ifndef MEP_PLAN_MIN_PAIRS_PER_TILE
+#define MEP_PLAN_MIN_PAIRS_PER_TILE 2048
+#endif
+constexpr int64_t kPlanMinPairsPerBlock = MEP_PLAN_MIN_PAIRS_PER_TILE;
 constexpr size_t kPlanWsHeader = 256;         // grid-barrier words
 
 size_t plan_workspace_bytes(const mep_shape_t &s);
