@@ -7,9 +7,9 @@
 // scaled by its router weight and to every router weight as the dot product
 // of the output gradient with the slot's expert output.
 //
-// One warp per token walks the row once in 16-byte chunks (lane l owns
-// chunks l, l+32, ...): it loads the output-gradient chunk and the K
-// expert-output chunks (all issued before use), accumulates the K partial dot
+// One warp per token walks the row once, kU 16-byte chunks per lane per step
+// (lane l owns chunks l, l+32, ...): it loads the output-gradient chunks and
+// the K expert-output chunks (all issued before use), accumulates the K partial dot
 // products in float32 FMAs, and stores the K scaled chunks.  The K partial
 // dots are summed across the warp with a fixed butterfly, so runs are
 // bit-identical.  The scaled gradient is rounded once: the float32 product is
@@ -27,6 +27,9 @@
 #ifndef MEP_COMBINE_BWD_BLOCKS_PER_SM
 #define MEP_COMBINE_BWD_BLOCKS_PER_SM 1024  // grid cap in multiples of the SM count
 #endif
+#ifndef MEP_COMBINE_BWD_U
+#define MEP_COMBINE_BWD_U 2  // 16-byte chunks per lane per iteration
+#endif
 
 namespace mep {
 
@@ -34,6 +37,7 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
+constexpr int kU = MEP_COMBINE_BWD_U;
 
 struct CombineBwdParams {
   const uint16_t *grad_out;
@@ -97,32 +101,44 @@ __global__ void __launch_bounds__(kThreads) combine_bwd_kernel(CombineBwdParams 
     // Warp-uniform loop over the row (every lane runs every iteration, so the
     // shuffles below always see the full warp); memory accesses are
     // predicated on the lane's chunk being inside the row.
-    for (int c0 = 0; c0 < p.chunks; c0 += 32) {
-      const int c = c0 + lane;
-      const bool in_row = c < p.chunks;
-      float gf[8];
-      unpack8(in_row ? __ldcs(gorow + c) : make_uint4(0, 0, 0, 0), gf);
+    for (int c0 = 0; c0 < p.chunks; c0 += 32 * kU) {
+      float gf[kU][8];
+      bool in_row[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int c = c0 + u * 32 + lane;
+        in_row[u] = c < p.chunks;
+        unpack8(in_row[u] ? __ldcs(gorow + c) : make_uint4(0, 0, 0, 0), gf[u]);
+      }
 #pragma unroll
       for (int kg = 0; kg < KC; kg += KG) {
-        uint4 yv[KG];
+        uint4 yv[KG][kU];
 #pragma unroll
         for (int j = 0; j < KG; ++j) {
           const int pk = __shfl_sync(0xffffffffu, sl, kg + j);
-          yv[j] = (in_row && ((okmask >> (kg + j)) & 1) && (unsigned)pk < (unsigned)p.NK)
-                      ? __ldcs(reinterpret_cast<const uint4 *>(p.y + (int64_t)pk * p.H) + c)
-                      : make_uint4(0, 0, 0, 0);
+          const bool ok = ((okmask >> (kg + j)) & 1) && (unsigned)pk < (unsigned)p.NK;
+          const uint4 *yrow = reinterpret_cast<const uint4 *>(p.y + (int64_t)(ok ? pk : 0) * p.H);
+#pragma unroll
+          for (int u = 0; u < kU; ++u)
+            yv[j][u] = (ok && in_row[u]) ? __ldcs(yrow + c0 + u * 32 + lane) : make_uint4(0, 0, 0, 0);
         }
 #pragma unroll
         for (int j = 0; j < KG; ++j) {
           const int k = kg + j;
           const int pk = __shfl_sync(0xffffffffu, sl, k);
           const float wk = __shfl_sync(0xffffffffu, wt, k);
-          if (in_row && ((okmask >> k) & 1) && (unsigned)pk < (unsigned)p.NK) {
-            float yf[8];
-            unpack8(yv[j], yf);
+          if (((okmask >> k) & 1) && (unsigned)pk < (unsigned)p.NK) {
+            uint4 *gyrow = reinterpret_cast<uint4 *>(p.grad_y + (int64_t)pk * p.H);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) dot[k] = __fmaf_rn(gf[e], yf[e], dot[k]);
-            __stcs(reinterpret_cast<uint4 *>(p.grad_y + (int64_t)pk * p.H) + c, scale8(wk, gf));
+            for (int u = 0; u < kU; ++u) {
+              if (in_row[u]) {
+                float yf[8];
+                unpack8(yv[j][u], yf);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) dot[k] = __fmaf_rn(gf[u][e], yf[e], dot[k]);
+                __stcs(gyrow + c0 + u * 32 + lane, scale8(wk, gf[u]));
+              }
+            }
           }
         }
       }
