@@ -8,10 +8,12 @@ mep_dispatch -> mep_combine -> mep_reduce_replica_grads, all through the C ABI.
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mep|reference]
 
 * value: tokens per second of the whole job (tokens of all ranks / max-over-ranks
-  device time), inputs resident in HBM, L2 flushed (512 MB write) between
-  steps outside the timed events.  The step is captured once in a CUDA graph
-  and replayed (``eager`` keeps the launch-by-launch timing, whose per-kernel
-  events give the roofline breakdown).
+  device time), inputs resident in HBM, L2 flushed between steps outside the
+  timed events (a 512 MB write, then a 512 MB read that writes the fill's
+  dirty lines back, so no timed kernel pays for the flush's write-back).  The
+  step is captured once in a CUDA graph and replayed (``eager`` keeps the
+  launch-by-launch timing, whose per-kernel events give the roofline
+  breakdown).
 * e2e: the same metric through the public API with pinned host buffers: every
   step copies that step's inputs host->device and its outputs (combine
   output, home gradients, plan scalars) back; consecutive steps overlap on
@@ -197,9 +199,6 @@ def oracle_throughput(wl, target_seconds: float, host=None):
         idx, w = workloads.routing(wl)
         host = dict(idx=idx, w=w)
     idx, w = host["idx"], host["w"]
-    t0 = time.perf_counter()
-    pl = ora.plan(R, S, E, K, idx)
-    t_plan = time.perf_counter() - t0
     # size the samples from the budget (about 12 ns per combine term, 3 ns per
     # reduced element on this kind of host core)
     per_tok = K * H * 12.5e-9
@@ -207,26 +206,37 @@ def oracle_throughput(wl, target_seconds: float, host=None):
     x = workloads.hidden(n_tok, H, seed=1).view(__import__("torch").int16).numpy().view(np.uint16)
     y = workloads.expert_outputs(n_tok * K, H, seed=2).view(__import__("torch").int16).numpy().view(np.uint16)
     pairs = np.arange(n_tok * K, dtype=np.int32)
-    t0 = time.perf_counter()
-    ora.dispatch(K, pairs, x)
-    t_disp = time.perf_counter() - t0
     local_slot = np.arange(n_tok * K, dtype=np.int32).reshape(n_tok, K)
-    t0 = time.perf_counter()
-    ora.combine(local_slot, w[:n_tok], y)
-    t_comb = time.perf_counter() - t0
-    t_red, n_col = 0.0, 0
-    if P:
-        n_col = int(max(1, min(P, (0.4 * target_seconds) / (3.2e-9 * (wl.seg_rows + E)))))
-        G = workloads.seg_grads(wl.seg_rows, n_col, seed=3).numpy()
+    n_col = int(max(1, min(P, (0.4 * target_seconds) / (3.2e-9 * (wl.seg_rows + E))))) if P else 0
+    G = workloads.seg_grads(wl.seg_rows, n_col, seed=3).numpy() if P else None
+    # Where the sample is the whole workload and takes less than the budget,
+    # it is repeated (at most 8 times) and the median repetition is reported.
+    reps, measured = [], 0.0
+    while not reps or (measured < 0.8 * target_seconds and len(reps) < 8):
         t0 = time.perf_counter()
-        ora.reduce(pl["expert_seg_ptr"], G)
-        t_red = time.perf_counter() - t0
-    t_step = t_plan + (t_disp + t_comb) * (N / n_tok) + (t_red * (P / n_col) if P else 0.0)
+        pl = ora.plan(R, S, E, K, idx)
+        t_plan = time.perf_counter() - t0
+        t0 = time.perf_counter()
+        ora.dispatch(K, pairs, x)
+        t_disp = time.perf_counter() - t0
+        t0 = time.perf_counter()
+        ora.combine(local_slot, w[:n_tok], y)
+        t_comb = time.perf_counter() - t0
+        t_red = 0.0
+        if P:
+            t0 = time.perf_counter()
+            ora.reduce(pl["expert_seg_ptr"], G)
+            t_red = time.perf_counter() - t0
+        t_step = t_plan + (t_disp + t_comb) * (N / n_tok) + (t_red * (P / n_col) if P else 0.0)
+        reps.append((t_step, dict(plan=t_plan, dispatch=t_disp, combine=t_comb, reduce=t_red)))
+        measured += t_plan + t_disp + t_comb + t_red
+    reps.sort(key=lambda r: r[0])
+    t_step, parts = reps[len(reps) // 2]
     sample = (f"whole plan; dispatch+combine of {n_tok}/{N} tokens; "
-              f"reduce of {n_col}/{P} gradient columns; scaled to the full step")
-    return dict(value=N / t_step, t_step=t_step, sample=sample,
-                measured_s=t_plan + t_disp + t_comb + t_red,
-                parts=dict(plan=t_plan, dispatch=t_disp, combine=t_comb, reduce=t_red))
+              f"reduce of {n_col}/{P} gradient columns; scaled to the full step; "
+              f"median of {len(reps)} repetition(s)")
+    return dict(value=N / t_step, t_step=t_step, sample=sample, measured_s=measured,
+                repetitions=len(reps), parts=parts)
 
 
 def run_reference(args):
@@ -294,6 +304,15 @@ def main():
     out = torch.empty((N, H), dtype=torch.bfloat16, device=dev)
     home = torch.empty((E, P), dtype=torch.float32, device=dev) if P else None
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    clean = torch.ones(FLUSH_BYTES // 8, dtype=torch.int64, device=dev)
+
+    def flush_l2():
+        # A write larger than L2 evicts every line of the step's inputs and
+        # outputs; the read of a second buffer larger than L2 then writes back
+        # the fill's own dirty lines, so the timed kernels start from a cold,
+        # clean L2 and pay for no one else's write-back.
+        flush.zero_()
+        clean.sum()
 
     def step(evs=None):
         if evs:
@@ -314,7 +333,7 @@ def main():
 
     launches_per_step = 4 if P else 3
     for _ in range(max(3, args.warmup)):
-        flush.zero_()
+        flush_l2()
         step()
     torch.cuda.synchronize()
     if mep.mep_read_status(plan) != 0:
@@ -327,7 +346,7 @@ def main():
         dist.barrier()
     torch.cuda.synchronize()
     for i in range(args.steps):
-        flush.zero_()
+        flush_l2()
         step(evs[i])
     torch.cuda.synchronize()
     if world > 1:
@@ -368,7 +387,7 @@ def main():
         hf = mep.Plan(s, dev)
         hts = []
         for it in range(3 + 20):
-            flush.zero_()
+            flush_l2()
             h0, h1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             h0.record()
             mep.mep_plan_home_first(s, idx, hf)
@@ -398,7 +417,7 @@ def main():
             step()
         gts = []
         for it in range(3 + args.steps):
-            flush.zero_()
+            flush_l2()
             g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             g0.record()
             cg.replay()
@@ -432,7 +451,7 @@ def main():
         for name, (fn, nbytes) in bwd.items():
             ts = []
             for it in range(3 + 20):
-                flush.zero_()
+                flush_l2()
                 b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 b0.record()
                 fn()
@@ -549,7 +568,8 @@ def main():
             "dtype": "bf16", "data": "synthetic",
             "config": {"workload": wl.name, "R": R, "S": S, "E": E, "K": K, "H": H, "P": P,
                        "step": "plan+dispatch+combine+replica-grad reduce",
-                       "l2": "flushed by a 512 MB write between steps, outside the events",
+                       "l2": ("flushed between steps, outside the events: a 512 MB write, then a "
+                              "512 MB read that writes the fill's dirty lines back"),
                        "timing": ("CUDA-graph replay of the captured step, events around each replay"
                                   if graph is not None else "eager launches, events around each kernel"),
                        "parallelism": f"replicas x{world}"},

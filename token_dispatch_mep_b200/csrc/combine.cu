@@ -13,9 +13,10 @@
 // order with one float32 FMA each, so every output is the same k-ordered
 // float32 sum whatever the grouping; the sum is rounded to bf16 and written
 // with a streaming 16-byte store.  Expert outputs are read once (streaming
-// loads).  The grid has one warp per token.  A form with warp tasks over
-// parts of rows and all K loads in flight measured 0.90-1.00 of the HBM copy
-// peak against 0.96-1.04 for this one.
+// loads).  The grid has one warp per token, in blocks of two warps: small
+// blocks keep the last wave short (1 % over blocks of eight warps).  A form
+// with warp tasks over parts of rows and all K loads in flight measured
+// 0.90-1.00 of the HBM copy peak against 0.96-1.04 for this one.
 //
 // Rank-addressed form (mep_combine_ranked): expert outputs are read from R
 // separate rank buffers, slot p being row p % SK of rank_ys[p / SK].
@@ -32,7 +33,7 @@
 #include "mep_internal.h"
 
 #ifndef MEP_COMBINE_MIN_BLOCKS
-#define MEP_COMBINE_MIN_BLOCKS 2  // launch bound: resident blocks per SM
+#define MEP_COMBINE_MIN_BLOCKS 8  // launch bound: resident blocks per SM
 #endif
 #ifndef MEP_COMBINE_ROW_U
 #define MEP_COMBINE_ROW_U 2  // 16-byte chunks per lane per step
@@ -42,7 +43,7 @@ namespace mep {
 
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 64;  // two token rows per block
 constexpr int kWarps = kThreads / 32;
 
 struct CombineParams {

@@ -35,8 +35,10 @@
 //            the same id) and the popcount of the peers below the lane.
 // A warp whose range exceeds its shared-memory id buffer reads its ids again
 // from global memory (L2 hits) in phase 3.
+#include <atomic>
 #include <climits>
 #include <cstdint>
+#include <mutex>
 
 #include "mep_device.cuh"
 #include "mep_internal.h"
@@ -490,13 +492,34 @@ __global__ void __launch_bounds__(kThreads, 1) plan_kernel(PlanParams p) {
   if (p.nb > 1) grid_barrier_exit(p.bar, p.nb);
 }
 
+// Per-device launch constants, shared by host threads.  The shared-memory
+// attribute only grows (a launch may ask for less than it allows), and
+// max_blocks is the co-resident block count at the largest size asked for,
+// a lower bound for every smaller one.  Updates hold the mutex; a launch whose
+// size is already allowed only reads the two atomics.
 struct PlanDev {
-  int sms = 0;
-  int max_blocks = 0;  // co-resident plan blocks (cooperative grid limit)
-  int smem_attr = -1;  // dynamic smem size the attribute was set for
+  std::mutex mu;
+  std::atomic<int> smem_attr{-1};  // largest dynamic shared memory allowed so far
+  std::atomic<int> max_blocks{0};  // co-resident plan blocks (cooperative grid limit)
 };
 
 PlanDev g_plan_dev[64];
+
+cudaError_t plan_dev_allow(PlanDev &d, int dev, int smem) {
+  std::lock_guard<std::mutex> lock(d.mu);
+  if (d.smem_attr.load(std::memory_order_acquire) >= smem) return cudaSuccess;
+  cudaError_t err = cudaFuncSetAttribute(plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (err != cudaSuccess) return err;
+  int sms = 0, per_sm = 0;
+  if ((err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+    return err;
+  err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, plan_kernel, kThreads, smem);
+  if (err != cudaSuccess) return err;
+  if (per_sm < 1) return cudaErrorInvalidConfiguration;
+  d.max_blocks.store(per_sm * sms, std::memory_order_relaxed);
+  d.smem_attr.store(smem, std::memory_order_release);
+  return cudaSuccess;
+}
 
 }  // namespace
 
@@ -512,22 +535,14 @@ cudaError_t launch_plan(const mep_shape_t &s, const int32_t *idx, const mep_plan
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   PlanDev &d = g_plan_dev[dev];
   const size_t smem = ((size_t)kWarps * s.E + (size_t)kWarps * kPlanIdsPerWarp) * sizeof(int);
-  if (d.smem_attr != (int)smem) {
-    err = cudaFuncSetAttribute(plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (err != cudaSuccess) return err;
-    err = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
-    if (err != cudaSuccess) return err;
-    int per_sm = 0;
-    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, plan_kernel, kThreads, smem);
-    if (err != cudaSuccess) return err;
-    if (per_sm < 1) return cudaErrorInvalidConfiguration;
-    d.max_blocks = per_sm * d.sms;
-    d.smem_attr = (int)smem;
-  }
+  if (d.smem_attr.load(std::memory_order_acquire) < (int)smem &&
+      (err = plan_dev_allow(d, dev, (int)smem)) != cudaSuccess)
+    return err;
+  const int max_blocks = d.max_blocks.load(std::memory_order_relaxed);
   const int64_t NK = (int64_t)s.R * s.S * s.K;
   int64_t want = (NK + kPlanMinPairsPerBlock - 1) / kPlanMinPairsPerBlock;
   // One block for a single tile; otherwise a coordinator plus nt tiles.
-  const int64_t cap = std::min(d.max_blocks, kPlanMaxBlocks) - 1;
+  const int64_t cap = std::min(max_blocks, kPlanMaxBlocks) - 1;
   const int nt = (int)std::max<int64_t>(1, std::min<int64_t>(want, cap));
   const int nb = nt > 1 ? nt + 1 : 1;
   PlanParams p{};
