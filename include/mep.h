@@ -65,7 +65,7 @@ extern "C" {
 #define MEP_API
 #endif
 
-#define MEP_VERSION 2
+#define MEP_VERSION 3
 #define MEP_MAX_EXPERTS 1024      /* E <= 1024 */
 #define MEP_MAX_RANKS 1024        /* R <= 1024 */
 #define MEP_MAX_HIDDEN 32768      /* H <= 32768 bf16 elements per row */
@@ -223,6 +223,86 @@ MEP_API mep_status_t mep_dispatch_ranked(mep_shape_t shape, int32_t H, const mep
 MEP_API mep_status_t mep_combine_ranked(mep_shape_t shape, int32_t H, const mep_plan_t *plan,
                                         const uint16_t *const *rank_ys, const float *topk_w,
                                         uint16_t *out, void *stream);
+
+/* One rank's share of the exchange: the rank-addressed dispatch and combine
+ * restricted to the tokens [token_begin, token_begin + token_count) of the
+ * global order -- on a multi-GPU system, the tokens this GPU holds (rank r:
+ * token_begin = r*S, token_count = S), after every rank has computed the same
+ * plan from the gathered router ids.  Row i of x, out and topk_w belongs to
+ * global token token_begin + i:
+ *   x       bf16 [token_count, H]   the local hidden rows (dispatch input).
+ *   topk_w  float32 [token_count, K] the local router weights (combine).
+ *   out     bf16 [token_count, H] out: the local combine output.
+ * rank_bufs / rank_ys as in mep_dispatch_ranked / mep_combine_ranked; every
+ * pointer in them must be non-NULL and 16-byte aligned (checked on the
+ * device: a bad one records MEP_ERR_DEVICE_DATA and is not dereferenced).
+ * 0 <= token_begin, 0 <= token_count, token_begin + token_count <= N, else
+ * MEP_ERR_INVALID_ARG; token_count == 0 is a no-op.  Calls over disjoint
+ * token ranges that cover [0, N) give exactly the results of the whole-range
+ * calls. */
+MEP_API mep_status_t mep_dispatch_ranked_tokens(mep_shape_t shape, int32_t H,
+                                                const mep_plan_t *plan, int64_t token_begin,
+                                                int64_t token_count, const uint16_t *x,
+                                                uint16_t *const *rank_bufs, void *stream);
+MEP_API mep_status_t mep_combine_ranked_tokens(mep_shape_t shape, int32_t H,
+                                               const mep_plan_t *plan, int64_t token_begin,
+                                               int64_t token_count,
+                                               const uint16_t *const *rank_ys,
+                                               const float *topk_w, uint16_t *out, void *stream);
+
+/* One home rank's share of the backward reduction ("How MoonEP works": the
+ * duplicates' gradients are summed into the home copy), with every rank's
+ * segment gradients in a buffer of its own.
+ *   home_rank   0 <= home_rank < R; its experts are e = home_rank*E/R ...
+ *               (home_rank+1)*E/R - 1.
+ *   rank_grads  device array of R device pointers (8-byte aligned); pointer r
+ *               addresses rank r's float32 rows [rank_rows, P], row j holding
+ *               the gradient of rank r's j-th segment in slot order, i.e.
+ *               segment rank_seg_idx[rank_seg_ptr[r] + j].  A rank holds at
+ *               most min(E, S*K) segments, so rank_rows = min(E, S*K) always
+ *               suffices.  Each pointer 16-byte aligned when P % 4 == 0 (else
+ *               4).  A NULL or misaligned pointer, or a segment at j >=
+ *               rank_rows, is detected on the device, records
+ *               MEP_ERR_DEVICE_DATA and contributes nothing.  Only the pointers
+ *               of ranks that hold a segment of a home expert are read.
+ *   rank_rows   rows of every rank's gradient buffer, >= 1.
+ *   home_grads  float32 [E/R, P] out: row i = sum over the segments of expert
+ *               home_rank*E/R + i, ascending segment index, in float32 (the
+ *               same sums, bit for bit, as rows of mep_reduce_replica_grads);
+ *               zero for an expert with no segment.
+ *   P >= 0; P == 0 is a no-op. */
+MEP_API mep_status_t mep_reduce_replica_grads_ranked(mep_shape_t shape, const mep_plan_t *plan,
+                                                     int64_t P, int32_t home_rank,
+                                                     const float *const *rank_grads,
+                                                     int64_t rank_rows, float *home_grads,
+                                                     void *stream);
+
+/* Buffer sharing between processes (one process per GPU): rank r exports its
+ * receive, expert-output and gradient buffers, the others map them and put
+ * the mapped addresses into the device pointer arrays above.  Host calls,
+ * synchronous, no kernel; CUDA IPC underneath, so the memory must come from
+ * cudaMalloc (directly or through a caching allocator of cudaMalloc
+ * segments).  Mapping and unmapping a peer's allocation is the only memory
+ * management in the library; it never allocates.
+ *   mep_ipc_export  describes [ptr, ptr + bytes) of the current device:
+ *                   `out` receives the allocation's IPC handle, the offset of
+ *                   ptr inside it and `bytes`.  MEP_ERR_INVALID_ARG if the
+ *                   range is not inside one allocation, MEP_ERR_CUDA if CUDA
+ *                   refuses the handle.
+ *   mep_ipc_open    in another process: maps the allocation (peer access
+ *                   enabled lazily) and returns the exported address in
+ *                   *ptr.  A process may not open its own export.
+ *   mep_ipc_close   unmaps what mep_ipc_open returned for the same handle;
+ *                   call after the last kernel that reads or writes it has
+ *                   finished. */
+typedef struct {
+    unsigned char handle[64];   /* cudaIpcMemHandle_t of the allocation */
+    uint64_t offset;            /* byte offset of the exported range in it */
+    uint64_t bytes;             /* length of the exported range */
+} mep_ipc_handle_t;
+MEP_API mep_status_t mep_ipc_export(const void *ptr, uint64_t bytes, mep_ipc_handle_t *out);
+MEP_API mep_status_t mep_ipc_open(const mep_ipc_handle_t *handle, void **ptr);
+MEP_API mep_status_t mep_ipc_close(const mep_ipc_handle_t *handle, void *ptr);
 
 /* Replica weight prefetch: before the expert compute, every replica gets a
  * copy of its expert's home weights ("How MoonEP works": the duplicates are

@@ -43,7 +43,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_version_and_strings(lib):
-    assert mep.mep_version() == 2
+    assert mep.mep_version() == 3
     for code, name in mep.STATUS.items():
         assert mep.mep_status_string(code)
     assert mep.mep_status_string(99) == "unknown status"
@@ -122,3 +122,52 @@ def test_package_has_no_cpu_fallback(tmp_path, monkeypatch):
     monkeypatch.setattr(mep, "_LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError):
         mep.load_library()
+
+
+def test_host_side_rejections_of_the_exchange_calls(lib):
+    """Token ranges, home ranks, NULL and misaligned pointers of the per-rank
+    exchange calls are rejected on the host; an empty range is a no-op."""
+    L = lib
+    s = mep.Shape(2, 4, 4, 2)           # N = 8 tokens
+    vp = ctypes.c_void_p
+    good = vp(0x100000)
+    p = _plan_struct()
+    pp = ctypes.byref(p)
+    # token ranges
+    for b, n in [(-1, 1), (0, -1), (0, 9), (8, 1), (9, 0), (4, 5)]:
+        assert L.mep_dispatch_ranked_tokens(s, 8, pp, b, n, good, good, None) == 1, (b, n)
+        assert L.mep_combine_ranked_tokens(s, 8, pp, b, n, good, good, good, None) == 1, (b, n)
+    for b in (0, 3, 8):
+        assert L.mep_dispatch_ranked_tokens(s, 8, pp, b, 0, None, None, None) == 0
+        assert L.mep_combine_ranked_tokens(s, 8, pp, b, 0, None, None, None, None) == 0
+    # NULL, misaligned, hidden size
+    assert L.mep_dispatch_ranked_tokens(s, 8, pp, 0, 4, None, good, None) == 1
+    assert L.mep_dispatch_ranked_tokens(s, 8, pp, 0, 4, good, None, None) == 1
+    assert L.mep_dispatch_ranked_tokens(s, 8, pp, 0, 4, vp(0x100008), good, None) == 2
+    assert L.mep_dispatch_ranked_tokens(s, 8, pp, 0, 4, good, vp(0x100004), None) == 2
+    assert L.mep_dispatch_ranked_tokens(s, 12, pp, 0, 4, good, good, None) == 2
+    assert L.mep_combine_ranked_tokens(s, 8, pp, 0, 4, good, None, good, None) == 1
+    assert L.mep_combine_ranked_tokens(s, 8, pp, 0, 4, good, good, vp(0x100008), None) == 2
+    # ranked reduce: home rank, P, pointers
+    for hr in (-1, 2):
+        assert L.mep_reduce_replica_grads_ranked(s, pp, 16, hr, good, 4, good, None) == 1
+    assert L.mep_reduce_replica_grads_ranked(s, pp, -1, 0, good, 4, good, None) == 1
+    assert L.mep_reduce_replica_grads_ranked(s, pp, 0, 0, None, 4, None, None) == 0
+    assert L.mep_reduce_replica_grads_ranked(s, pp, 16, 0, None, 4, good, None) == 1
+    assert L.mep_reduce_replica_grads_ranked(s, pp, 16, 0, good, 0, good, None) == 1
+    assert L.mep_reduce_replica_grads_ranked(s, pp, 16, 0, good, 4, None, None) == 1
+    assert L.mep_reduce_replica_grads_ranked(s, pp, 16, 0, vp(0x100004), 4, good, None) == 2
+    assert L.mep_reduce_replica_grads_ranked(s, pp, 16, 0, good, 4, vp(0x100004), None) == 2
+    q = _plan_struct()
+    q.rank_seg_idx = None
+    assert L.mep_reduce_replica_grads_ranked(s, ctypes.byref(q), 16, 0, good, 4, good, None) == 1
+    # IPC: NULL arguments never reach CUDA
+    h = mep.IpcHandle()
+    assert L.mep_ipc_export(None, 16, ctypes.byref(h)) == 1
+    assert L.mep_ipc_export(good, 0, ctypes.byref(h)) == 1
+    assert L.mep_ipc_export(good, 16, None) == 1
+    out = vp()
+    assert L.mep_ipc_open(None, ctypes.byref(out)) == 1
+    assert L.mep_ipc_open(ctypes.byref(h), None) == 1
+    assert L.mep_ipc_close(None, good) == 1
+    assert L.mep_ipc_close(ctypes.byref(h), None) == 1

@@ -83,7 +83,33 @@ def _case_sharded_plan(rank, world):
     return bool(np.array_equal(slots, want)), int(T.sum())
 
 
-CASES = {"max": _case_max, "sharded_plan": _case_sharded_plan}
+def _case_gather_ids(rank, world):
+    """ep.gather_router_ids over gloo: every rank ends with all ranks' ids in
+    global token order, and the oracle plan of them gives each rank a
+    segment list (ep.local_segments) that covers its S*K slots in order."""
+    import torch
+
+    import oracle
+    from token_dispatch_mep_b200 import ep
+    R, S, E, K = world, 257, 16, 3
+    rng = np.random.default_rng(7)
+    logits = rng.standard_normal((R * S, E)) - 1.1 * np.log(np.arange(1, E + 1))
+    idx = np.argsort(-logits, axis=1, kind="stable")[:, :K].astype(np.int32)
+    got = ep.gather_router_ids(torch.from_numpy(idx[rank * S:(rank + 1) * S].copy()))
+    same = bool(np.array_equal(got.numpy(), idx))
+    covered = []
+    for plan in (oracle.get().plan(R, S, E, K, idx), oracle.get().plan_home_first(R, S, E, K, idx)):
+        segs = ep.local_segments(plan, rank)
+        starts = [st for _, _, st, _ in segs]
+        experts = [e for _, e, _, _ in segs]
+        covered.append((sum(c for _, _, _, c in segs) == S * K,
+                        starts == sorted(starts) and (not starts or starts[0] == 0),
+                        len(segs) <= ep.max_local_segments(type("Sh", (), dict(E=E, SK=S * K))()),
+                        len(set(experts)) == len(experts)))
+    return same, covered
+
+
+CASES = {"max": _case_max, "sharded_plan": _case_sharded_plan, "gather_ids": _case_gather_ids}
 
 
 def _run(case, world=2):
@@ -125,3 +151,12 @@ def test_reference_arm_prints_on_rank_zero_only(monkeypatch):
     with redirect_stdout(buf):
         bench.run_reference(args)
     assert buf.getvalue() == ""
+
+
+def test_router_id_gather_and_local_segment_lists():
+    out = _run("gather_ids")
+    for rank in (0, 1):
+        same, covered = out[rank]
+        assert same is True, out
+        for flags in covered:                   # contiguous, home-first
+            assert all(flags), (rank, flags)

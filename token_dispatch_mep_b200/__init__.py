@@ -21,7 +21,9 @@ __all__ = [
     "mep_plan_workspace_bytes", "mep_maxvio", "mep_plan", "mep_plan_home_first", "mep_plan_noalloc",
     "mep_dispatch",
     "mep_combine", "mep_combine_backward", "mep_dispatch_backward", "mep_prefetch_replica_weights",
-    "mep_dispatch_ranked", "mep_combine_ranked", "rank_pointer_table",
+    "mep_dispatch_ranked", "mep_combine_ranked", "rank_pointer_table", "pointer_table",
+    "mep_dispatch_ranked_tokens", "mep_combine_ranked_tokens", "mep_reduce_replica_grads_ranked",
+    "IpcHandle", "mep_ipc_export", "mep_ipc_open", "mep_ipc_close",
     "mep_reduce_replica_grads", "mep_read_status", "mep_status_string",
     "mep_set_wait_limit_ns", "mep_get_wait_limit_ns", "mep_version", "STATUS",
 ]
@@ -38,7 +40,9 @@ ABI_SYMBOLS = ("mep_plan_workspace_bytes", "mep_maxvio", "mep_plan", "mep_dispat
                "mep_set_wait_limit_ns", "mep_get_wait_limit_ns", "mep_version",
                "mep_plan_noalloc", "mep_combine_backward", "mep_dispatch_backward",
                "mep_prefetch_replica_weights", "mep_plan_home_first", "mep_dispatch_ranked",
-               "mep_combine_ranked")
+               "mep_combine_ranked", "mep_dispatch_ranked_tokens", "mep_combine_ranked_tokens",
+               "mep_reduce_replica_grads_ranked", "mep_ipc_export", "mep_ipc_open",
+               "mep_ipc_close")
 
 
 class MepError(RuntimeError):
@@ -70,6 +74,14 @@ class Shape(ctypes.Structure):
 
     def __repr__(self):
         return f"Shape(R={self.R}, S={self.S}, E={self.E}, K={self.K})"
+
+
+class IpcHandle(ctypes.Structure):
+    """``mep_ipc_handle_t``: a CUDA IPC handle of an allocation, the exported
+    range's offset in it and its length.  ``bytes(h)`` / ``IpcHandle.from_buffer_copy``
+    move it between processes."""
+    _fields_ = [("handle", ctypes.c_ubyte * 64), ("offset", ctypes.c_uint64),
+                ("bytes", ctypes.c_uint64)]
 
 
 class _PlanStruct(ctypes.Structure):
@@ -116,6 +128,12 @@ def load_library():
         "mep_plan_home_first": ([Shape, vp, P, vp, sz, vp], ctypes.c_int),
         "mep_dispatch_ranked": ([Shape, i32, P, vp, vp, vp], ctypes.c_int),
         "mep_combine_ranked": ([Shape, i32, P, vp, vp, vp, vp], ctypes.c_int),
+        "mep_dispatch_ranked_tokens": ([Shape, i32, P, i64, i64, vp, vp, vp], ctypes.c_int),
+        "mep_combine_ranked_tokens": ([Shape, i32, P, i64, i64, vp, vp, vp, vp], ctypes.c_int),
+        "mep_reduce_replica_grads_ranked": ([Shape, P, i64, i32, vp, i64, vp, vp], ctypes.c_int),
+        "mep_ipc_export": ([vp, u64, ctypes.POINTER(IpcHandle)], ctypes.c_int),
+        "mep_ipc_open": ([ctypes.POINTER(IpcHandle), ctypes.POINTER(vp)], ctypes.c_int),
+        "mep_ipc_close": ([ctypes.POINTER(IpcHandle), vp], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -349,6 +367,88 @@ def mep_combine_ranked(shape, H: int, plan: Plan, rank_table, topk_w, out):
     op = _need(out, "out", torch.bfloat16, s.N * H, dev)
     _ok(L.mep_combine_ranked(s, int(H), ctypes.byref(plan.struct), tp, wp, op, _stream(dev)),
         "mep_combine_ranked")
+
+
+def pointer_table(ptrs, device) -> torch.Tensor:
+    """Device array of raw device addresses (e.g. peers' buffers mapped by
+    ``mep_ipc_open``), for the rank-addressed calls."""
+    return torch.tensor([int(p) for p in ptrs], dtype=torch.int64, device=device)
+
+
+def _token_range(s: Shape, token_begin: int, token_count: int):
+    if token_begin < 0 or token_count < 0 or token_begin + token_count > s.N:
+        raise ValueError(f"token range [{token_begin}, {token_begin + token_count}) outside [0, {s.N})")
+
+
+def mep_dispatch_ranked_tokens(shape, H: int, plan: Plan, token_begin: int, x, rank_table,
+                               token_count: int | None = None):
+    """Dispatch of the tokens [token_begin, token_begin + token_count) (default:
+    all rows of ``x``) into R rank buffers; ``x`` holds those tokens' rows."""
+    L, s = load_library(), _shape(shape)
+    dev = plan.device
+    n = x.shape[0] if token_count is None else int(token_count)
+    _token_range(s, int(token_begin), n)
+    xp = _need(x, "x", torch.bfloat16, n * H, dev)
+    tp = _need(rank_table, "rank_table", torch.int64, s.R, dev)
+    _ok(L.mep_dispatch_ranked_tokens(s, int(H), ctypes.byref(plan.struct), int(token_begin), n,
+                                     xp, tp, _stream(dev)), "mep_dispatch_ranked_tokens")
+
+
+def mep_combine_ranked_tokens(shape, H: int, plan: Plan, token_begin: int, rank_table, topk_w,
+                              out, token_count: int | None = None):
+    """Combine of the tokens [token_begin, token_begin + token_count) (default:
+    all rows of ``out``) from R rank buffers; ``topk_w`` and ``out`` hold those
+    tokens' rows."""
+    L, s = load_library(), _shape(shape)
+    dev = plan.device
+    n = out.shape[0] if token_count is None else int(token_count)
+    _token_range(s, int(token_begin), n)
+    tp = _need(rank_table, "rank_table", torch.int64, s.R, dev)
+    wp = _need(topk_w, "topk_w", torch.float32, n * s.K, dev)
+    op = _need(out, "out", torch.bfloat16, n * H, dev)
+    _ok(L.mep_combine_ranked_tokens(s, int(H), ctypes.byref(plan.struct), int(token_begin), n,
+                                    tp, wp, op, _stream(dev)), "mep_combine_ranked_tokens")
+
+
+def mep_reduce_replica_grads_ranked(shape, plan: Plan, P: int, home_rank: int, rank_table,
+                                    rank_rows: int, home_grads):
+    """Home rank ``home_rank``'s share of the replica-gradient reduction: rank
+    r's segment gradients are the ``rank_rows`` rows of the buffer at
+    ``rank_table[r]``, in r's slot order; ``home_grads`` fp32 [E/R, P]."""
+    L, s = load_library(), _shape(shape)
+    dev = plan.device
+    tp = _need(rank_table, "rank_table", torch.int64, s.R, dev)
+    hp = _need(home_grads, "home_grads", torch.float32, (s.E // s.R) * P, dev)
+    _ok(L.mep_reduce_replica_grads_ranked(s, ctypes.byref(plan.struct), int(P), int(home_rank),
+                                          tp, int(rank_rows), hp, _stream(dev)),
+        "mep_reduce_replica_grads_ranked")
+
+
+def mep_ipc_export(t: torch.Tensor) -> IpcHandle:
+    """IPC description of the CUDA tensor ``t``'s memory (contiguous)."""
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError("mep_ipc_export needs a contiguous CUDA tensor")
+    h = IpcHandle()
+    with torch.cuda.device(t.device):
+        _ok(load_library().mep_ipc_export(ctypes.c_void_p(t.data_ptr()),
+                                          t.numel() * t.element_size(), ctypes.byref(h)),
+            "mep_ipc_export")
+    return h
+
+
+def mep_ipc_open(h: IpcHandle, device) -> int:
+    """Map another process's exported range on ``device``; returns its address."""
+    p = ctypes.c_void_p()
+    with torch.cuda.device(torch.device(device)):
+        _ok(load_library().mep_ipc_open(ctypes.byref(h), ctypes.byref(p)), "mep_ipc_open")
+    return int(p.value)
+
+
+def mep_ipc_close(h: IpcHandle, ptr: int, device):
+    """Unmap what ``mep_ipc_open`` returned for ``h``."""
+    with torch.cuda.device(torch.device(device)):
+        _ok(load_library().mep_ipc_close(ctypes.byref(h), ctypes.c_void_p(int(ptr))),
+            "mep_ipc_close")
 
 
 def mep_reduce_replica_grads(shape, plan: Plan, P: int, seg_grads, home_grads):

@@ -36,6 +36,12 @@ mep_status_t check_ws(const mep_shape_t &s, const void *ws, size_t ws_bytes) {
   return MEP_OK;
 }
 
+mep_status_t check_tokens(const mep_shape_t &s, int64_t begin, int64_t count) {
+  const int64_t N = (int64_t)s.R * s.S;
+  if (begin < 0 || count < 0 || begin > N || count > N - begin) return MEP_ERR_INVALID_ARG;
+  return MEP_OK;
+}
+
 mep_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? MEP_OK : MEP_ERR_CUDA; }
 
 cudaStream_t as_stream(void *s) { return static_cast<cudaStream_t>(s); }
@@ -109,7 +115,8 @@ mep_status_t mep_dispatch(mep_shape_t shape, int32_t H, const mep_plan_t *plan, 
   if ((st = check_hidden(H)) != MEP_OK) return st;
   if (!plan || !plan->slot || !plan->status || !x || !buf) return MEP_ERR_INVALID_ARG;
   if (!aligned(x, 16) || !aligned(buf, 16) || !aligned(plan->slot, 4)) return MEP_ERR_MISALIGNED;
-  return from_cuda(mep::launch_dispatch(shape, H, *plan, x, buf, nullptr, as_stream(stream)));
+  return from_cuda(mep::launch_dispatch(shape, H, *plan, 0, (int64_t)shape.R * shape.S, x, buf,
+                                        nullptr, as_stream(stream)));
 }
 
 mep_status_t mep_combine(mep_shape_t shape, int32_t H, const mep_plan_t *plan, const uint16_t *y,
@@ -120,7 +127,8 @@ mep_status_t mep_combine(mep_shape_t shape, int32_t H, const mep_plan_t *plan, c
   if (!plan || !plan->slot || !plan->status || !y || !topk_w || !out) return MEP_ERR_INVALID_ARG;
   if (!aligned(y, 16) || !aligned(out, 16) || !aligned(topk_w, 4) || !aligned(plan->slot, 4))
     return MEP_ERR_MISALIGNED;
-  return from_cuda(mep::launch_combine(shape, H, *plan, y, nullptr, topk_w, out, as_stream(stream)));
+  return from_cuda(mep::launch_combine(shape, H, *plan, 0, (int64_t)shape.R * shape.S, y, nullptr,
+                                       topk_w, out, as_stream(stream)));
 }
 
 mep_status_t mep_reduce_replica_grads(mep_shape_t shape, const mep_plan_t *plan, int64_t P,
@@ -162,7 +170,8 @@ mep_status_t mep_dispatch_backward(mep_shape_t shape, int32_t H, const mep_plan_
   if (!aligned(grad_buf, 16) || !aligned(grad_x, 16) || !aligned(plan->slot, 4))
     return MEP_ERR_MISALIGNED;
   return from_cuda(
-      mep::launch_combine(shape, H, *plan, grad_buf, nullptr, nullptr, grad_x, as_stream(stream)));
+      mep::launch_combine(shape, H, *plan, 0, (int64_t)shape.R * shape.S, grad_buf, nullptr, nullptr,
+                          grad_x, as_stream(stream)));
 }
 
 mep_status_t mep_prefetch_replica_weights(mep_shape_t shape, const mep_plan_t *plan,
@@ -188,7 +197,23 @@ mep_status_t mep_dispatch_ranked(mep_shape_t shape, int32_t H, const mep_plan_t 
   if ((st = check_hidden(H)) != MEP_OK) return st;
   if (!plan || !plan->slot || !plan->status || !x || !rank_bufs) return MEP_ERR_INVALID_ARG;
   if (!aligned(x, 16) || !aligned(rank_bufs, 8) || !aligned(plan->slot, 4)) return MEP_ERR_MISALIGNED;
-  return from_cuda(mep::launch_dispatch(shape, H, *plan, x, nullptr, rank_bufs, as_stream(stream)));
+  return from_cuda(mep::launch_dispatch(shape, H, *plan, 0, (int64_t)shape.R * shape.S, x, nullptr,
+                                        rank_bufs, as_stream(stream)));
+}
+
+mep_status_t mep_dispatch_ranked_tokens(mep_shape_t shape, int32_t H, const mep_plan_t *plan,
+                                        int64_t token_begin, int64_t token_count,
+                                        const uint16_t *x, uint16_t *const *rank_bufs,
+                                        void *stream) {
+  mep_status_t st = check_shape(shape);
+  if (st != MEP_OK) return st;
+  if ((st = check_hidden(H)) != MEP_OK) return st;
+  if ((st = check_tokens(shape, token_begin, token_count)) != MEP_OK) return st;
+  if (token_count == 0) return MEP_OK;
+  if (!plan || !plan->slot || !plan->status || !x || !rank_bufs) return MEP_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(rank_bufs, 8) || !aligned(plan->slot, 4)) return MEP_ERR_MISALIGNED;
+  return from_cuda(mep::launch_dispatch(shape, H, *plan, token_begin, token_count, x, nullptr,
+                                        rank_bufs, as_stream(stream)));
 }
 
 mep_status_t mep_combine_ranked(mep_shape_t shape, int32_t H, const mep_plan_t *plan,
@@ -201,7 +226,45 @@ mep_status_t mep_combine_ranked(mep_shape_t shape, int32_t H, const mep_plan_t *
     return MEP_ERR_INVALID_ARG;
   if (!aligned(rank_ys, 8) || !aligned(out, 16) || !aligned(topk_w, 4) || !aligned(plan->slot, 4))
     return MEP_ERR_MISALIGNED;
-  return from_cuda(mep::launch_combine(shape, H, *plan, nullptr, rank_ys, topk_w, out, as_stream(stream)));
+  return from_cuda(mep::launch_combine(shape, H, *plan, 0, (int64_t)shape.R * shape.S, nullptr,
+                                       rank_ys, topk_w, out, as_stream(stream)));
+}
+
+mep_status_t mep_combine_ranked_tokens(mep_shape_t shape, int32_t H, const mep_plan_t *plan,
+                                       int64_t token_begin, int64_t token_count,
+                                       const uint16_t *const *rank_ys, const float *topk_w,
+                                       uint16_t *out, void *stream) {
+  mep_status_t st = check_shape(shape);
+  if (st != MEP_OK) return st;
+  if ((st = check_hidden(H)) != MEP_OK) return st;
+  if ((st = check_tokens(shape, token_begin, token_count)) != MEP_OK) return st;
+  if (token_count == 0) return MEP_OK;
+  if (!plan || !plan->slot || !plan->status || !rank_ys || !topk_w || !out)
+    return MEP_ERR_INVALID_ARG;
+  if (!aligned(rank_ys, 8) || !aligned(out, 16) || !aligned(topk_w, 4) || !aligned(plan->slot, 4))
+    return MEP_ERR_MISALIGNED;
+  return from_cuda(mep::launch_combine(shape, H, *plan, token_begin, token_count, nullptr, rank_ys,
+                                       topk_w, out, as_stream(stream)));
+}
+
+mep_status_t mep_reduce_replica_grads_ranked(mep_shape_t shape, const mep_plan_t *plan, int64_t P,
+                                             int32_t home_rank, const float *const *rank_grads,
+                                             int64_t rank_rows, float *home_grads, void *stream) {
+  mep_status_t st = check_shape(shape);
+  if (st != MEP_OK) return st;
+  if (P < 0 || !plan || home_rank < 0 || home_rank >= shape.R || rank_rows < 1)
+    return MEP_ERR_INVALID_ARG;
+  if (P == 0) return MEP_OK;
+  if (!plan->expert_seg_ptr || !plan->seg || !plan->rank_seg_ptr || !plan->rank_seg_idx ||
+      !plan->status || !rank_grads || !home_grads)
+    return MEP_ERR_INVALID_ARG;
+  if ((int64_t)shape.E * P > ((int64_t)1 << 46)) return MEP_ERR_INVALID_ARG;
+  const size_t a = (P % 4 == 0) ? 16 : 4;
+  if (!aligned(home_grads, a) || !aligned(rank_grads, 8) || !aligned(plan->expert_seg_ptr, 4) ||
+      !aligned(plan->seg, 16) || !aligned(plan->rank_seg_ptr, 4) || !aligned(plan->rank_seg_idx, 4))
+    return MEP_ERR_MISALIGNED;
+  return from_cuda(mep::launch_reduce_ranked(shape, *plan, P, home_rank, rank_grads, rank_rows,
+                                             home_grads, as_stream(stream)));
 }
 
 mep_status_t mep_read_status(const mep_plan_t *plan, void *stream) {

@@ -54,7 +54,8 @@ struct CombineParams {
   const int32_t *slot;
   uint16_t *out;
   int32_t *status;
-  int64_t N, NK;
+  int64_t g0;     // first token (global order); out / w row i is token g0 + i
+  int64_t N, NK;  // tokens processed, slots of the plan
   int32_t K, H;
   int32_t chunks;      // 16-byte chunks per row = H / 8
 };
@@ -88,7 +89,7 @@ __global__ void __launch_bounds__(kThreads, MEP_COMBINE_MIN_BLOCKS) combine_row_
   const int64_t nwarps = (int64_t)gridDim.x * kWarps;
   bool bad = false;
   for (int64_t g = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5); g < p.N; g += nwarps) {
-    int sl = lane < p.K ? __ldg(p.slot + g * p.K + lane) : -1;
+    int sl = lane < p.K ? __ldg(p.slot + (p.g0 + g) * p.K + lane) : -1;
     const float wt = lane < p.K ? (p.w != nullptr ? __ldg(p.w + g * p.K + lane) : 1.f) : 0.f;
     if (lane < p.K && (unsigned)sl >= (unsigned)p.NK) {
       bad = true;
@@ -108,12 +109,18 @@ __global__ void __launch_bounds__(kThreads, MEP_COMBINE_MIN_BLOCKS) combine_row_
 #pragma unroll
         for (int j = 0; j < KG; ++j) {
           const int pk = __shfl_sync(0xffffffffu, sl, kg + j);
-          const bool ok = ((okmask >> (kg + j)) & 1) && (unsigned)pk < (unsigned)p.NK;
+          bool ok = ((okmask >> (kg + j)) & 1) && (unsigned)pk < (unsigned)p.NK;
           const int64_t pp = ok ? pk : 0;
           const uint16_t *yrow;
           if (kRanked) {
+            // a rank buffer must be present and 16-byte aligned
             const int64_t r = pp / p.SK;
-            yrow = p.rank_ys[r] + (pp - r * p.SK) * p.H;
+            const uint16_t *base = p.rank_ys[r];
+            if (base == nullptr || (reinterpret_cast<uintptr_t>(base) & 15) != 0) {
+              if (ok) bad = true;
+              ok = false;
+            }
+            yrow = base + (pp - r * p.SK) * p.H;
           } else {
             yrow = p.y + pp * p.H;
           }
@@ -156,9 +163,10 @@ cudaError_t launch_kc(const CombineParams &p, int sms, cudaStream_t stream) {
 
 }  // namespace
 
-cudaError_t launch_combine(const mep_shape_t &s, int32_t H, const mep_plan_t &pl,
-                           const uint16_t *y, const uint16_t *const *rank_ys, const float *w,
-                           uint16_t *out, cudaStream_t stream) {
+cudaError_t launch_combine(const mep_shape_t &s, int32_t H, const mep_plan_t &pl, int64_t g0,
+                           int64_t count, const uint16_t *y, const uint16_t *const *rank_ys,
+                           const float *w, uint16_t *out, cudaStream_t stream) {
+  if (count <= 0) return cudaSuccess;
   int dev = 0, sms = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
@@ -172,8 +180,9 @@ cudaError_t launch_combine(const mep_shape_t &s, int32_t H, const mep_plan_t &pl
   p.slot = pl.slot;
   p.out = out;
   p.status = pl.status;
-  p.N = (int64_t)s.R * s.S;
-  p.NK = p.N * s.K;
+  p.g0 = g0;
+  p.N = count;
+  p.NK = (int64_t)s.R * s.S * s.K;
   p.K = s.K;
   p.H = H;
   p.chunks = H / 8;

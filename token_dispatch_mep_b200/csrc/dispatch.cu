@@ -64,7 +64,8 @@ struct DispatchParams {
   int64_t SK;
   const int32_t *slot;
   int32_t *status;
-  int64_t N, NK;
+  int64_t g0;     // first token (global order); x row i is token g0 + i
+  int64_t N, NK;  // tokens processed, slots of the plan
   int32_t K, H;
   int32_t chunks;  // 16-byte chunks per row = H / 8
   int32_t parts;   // warp tasks per token
@@ -78,7 +79,7 @@ __global__ void __launch_bounds__(kThreads) dispatch_kernel(DispatchParams p) {
   int64_t task = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
   bool bad = false;
   auto fetch = [&](int64_t t) -> int {
-    return (t < ntask && lane < p.K) ? __ldg(p.slot + (t / p.parts) * p.K + lane) : -1;
+    return (t < ntask && lane < p.K) ? __ldg(p.slot + (p.g0 + t / p.parts) * p.K + lane) : -1;
   };
   int sl = fetch(task);
   for (; task < ntask; task += nwarps) {
@@ -96,14 +97,19 @@ __global__ void __launch_bounds__(kThreads) dispatch_kernel(DispatchParams p) {
     for (int k = 0; k < KC; ++k) {
       const int pk = __shfl_sync(0xffffffffu, sl, k);
       if (k < p.K) {
+        uint16_t *row = nullptr;
         if ((unsigned)pk < (unsigned)p.NK) {
-          uint16_t *row;
           if (kRanked) {
+            // a rank buffer must be present and 16-byte aligned
             const int64_t r = pk / p.SK;
-            row = p.rank_bufs[r] + (pk - r * p.SK) * p.H;
+            uint16_t *base = p.rank_bufs[r];
+            if (base != nullptr && (reinterpret_cast<uintptr_t>(base) & 15) == 0)
+              row = base + (pk - r * p.SK) * p.H;
           } else {
             row = p.buf + (int64_t)pk * p.H;
           }
+        }
+        if (row != nullptr) {
           uint4 *brow = reinterpret_cast<uint4 *>(row);
 #pragma unroll
           for (int u = 0; u < kU; ++u) {
@@ -188,9 +194,10 @@ cudaError_t launch_kc(const DispatchParams &p, const DispatchDev &d, cudaStream_
 
 }  // namespace
 
-cudaError_t launch_dispatch(const mep_shape_t &s, int32_t H, const mep_plan_t &pl,
-                            const uint16_t *x, uint16_t *buf, uint16_t *const *rank_bufs,
-                            cudaStream_t stream) {
+cudaError_t launch_dispatch(const mep_shape_t &s, int32_t H, const mep_plan_t &pl, int64_t g0,
+                            int64_t count, const uint16_t *x, uint16_t *buf,
+                            uint16_t *const *rank_bufs, cudaStream_t stream) {
+  if (count <= 0) return cudaSuccess;
   DispatchDev *d = nullptr;
   const cudaError_t err = dispatch_dev(d);
   if (err != cudaSuccess) return err;
@@ -201,8 +208,9 @@ cudaError_t launch_dispatch(const mep_shape_t &s, int32_t H, const mep_plan_t &p
   p.SK = (int64_t)s.S * s.K;
   p.slot = pl.slot;
   p.status = pl.status;
-  p.N = (int64_t)s.R * s.S;
-  p.NK = p.N * s.K;
+  p.g0 = g0;
+  p.N = count;
+  p.NK = (int64_t)s.R * s.S * s.K;
   p.K = s.K;
   p.H = H;
   p.chunks = H / 8;

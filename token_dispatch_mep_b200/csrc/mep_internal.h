@@ -29,17 +29,25 @@ cudaError_t launch_plan(const mep_shape_t &s, const int32_t *idx, const mep_plan
                         int full, int kind, void *ws, uint64_t wait_ns, cudaStream_t stream);
 
 // rank_bufs / rank_ys: nullptr for one [R, S*K, H] buffer, else a device array
-// of R row buffers of S*K rows each.
-cudaError_t launch_dispatch(const mep_shape_t &s, int32_t H, const mep_plan_t &pl,
-                            const uint16_t *x, uint16_t *buf, uint16_t *const *rank_bufs,
-                            cudaStream_t stream);
+// of R row buffers of S*K rows each.  Tokens [g0, g0 + count) of the global
+// order are processed; row i of x / out and of w belongs to token g0 + i.
+cudaError_t launch_dispatch(const mep_shape_t &s, int32_t H, const mep_plan_t &pl, int64_t g0,
+                            int64_t count, const uint16_t *x, uint16_t *buf,
+                            uint16_t *const *rank_bufs, cudaStream_t stream);
 
-cudaError_t launch_combine(const mep_shape_t &s, int32_t H, const mep_plan_t &pl,
-                           const uint16_t *y, const uint16_t *const *rank_ys, const float *w,
-                           uint16_t *out, cudaStream_t stream);
+cudaError_t launch_combine(const mep_shape_t &s, int32_t H, const mep_plan_t &pl, int64_t g0,
+                           int64_t count, const uint16_t *y, const uint16_t *const *rank_ys,
+                           const float *w, uint16_t *out, cudaStream_t stream);
 
 cudaError_t launch_reduce(const mep_shape_t &s, const mep_plan_t &pl, int64_t P,
                           const float *G, float *home, cudaStream_t stream);
+
+// Home rank `home_rank`'s experts only: segment s is row j of rank_G[r], r its
+// rank and j its position in r's segment list (rank_seg_idx), j < rank_rows;
+// home holds the E/R rows of experts home_rank*E/R ...
+cudaError_t launch_reduce_ranked(const mep_shape_t &s, const mep_plan_t &pl, int64_t P,
+                                 int32_t home_rank, const float *const *rank_G,
+                                 int64_t rank_rows, float *home, cudaStream_t stream);
 
 cudaError_t launch_prefetch(const mep_shape_t &s, const mep_plan_t &pl, int64_t row_bytes,
                             const void *w_home, void *w_rep, cudaStream_t stream);

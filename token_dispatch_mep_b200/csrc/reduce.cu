@@ -16,6 +16,14 @@
 // both with streaming (evict-first) accesses.  The segment pointers are read
 // on the device and bounds-checked; nothing is sized from a host copy of the
 // plan.
+//
+// Rank-addressed form (mep_reduce_replica_grads_ranked): the gradients of a
+// rank's segments live in that rank's own buffer (on a multi-GPU system, a
+// peer buffer mapped into this GPU's address space), row j of rank r's
+// buffer holding the j-th segment of rank r's list in slot order.  One home
+// rank reduces its own E/R experts: for each task the block first resolves
+// the expert's segments to row addresses (segment -> rank -> position in
+// that rank's list, into shared memory), then sums exactly as above.
 #include <algorithm>
 #include <cstdint>
 
@@ -51,7 +59,18 @@ struct ReduceParams {
   int32_t E;
   int32_t rows;   // E + R - 1
   int64_t cols;   // P / 4 (vector path) or P (scalar path)
+  // ranked form
+  const float *const *rank_G;   // [R] rank gradient buffers
+  const int4 *seg;              // segments {expert, rank, start, count}
+  const int32_t *rank_seg_ptr;  // [R+1]
+  const int32_t *rank_seg_idx;  // [E+R-1] segment indices, rank by rank, slot order
+  int64_t rank_rows;            // rows of every rank gradient buffer
+  int32_t R;
+  int32_t e0;                   // first expert reduced (home rank * E/R)
+  int32_t ne;                   // experts reduced
 };
+
+constexpr int kMaxSegPerExpert = MEP_MAX_RANKS;  // an expert has at most one segment per rank
 
 template <typename V>
 __device__ __forceinline__ V zero_v();
@@ -65,21 +84,67 @@ __device__ __forceinline__ float4 addv(float4 a, float4 b) {
 }
 __device__ __forceinline__ float addv(float a, float b) { return a + b; }
 
+// Address of segment s's gradient row: row s of G, or (ranked form) the row
+// resolved into s_rows for this task (nullptr if it could not be resolved).
+template <typename V, bool kRanked>
+__device__ __forceinline__ const V *seg_row(const ReduceParams &p, const V *G,
+                                            const V *const *s_rows, int s, int s0) {
+  if (kRanked) return s_rows[s - s0];
+  return G + (int64_t)s * p.cols;
+}
+
+// Ranked form: threads t < s1 - s0 resolve segment s0 + t to its row in its
+// rank's buffer.  Returns false if any segment's data was out of range.
 template <typename V>
+__device__ bool resolve_rows(const ReduceParams &p, int s0, int s1, const V **s_rows) {
+  bool ok = true;
+  for (int t = threadIdx.x; t < s1 - s0; t += blockDim.x) {
+    const int s = s0 + t;
+    const V *row = nullptr;
+    const int r = __ldg(&p.seg[s].y);
+    if (r >= 0 && r < p.R) {
+      const int b = __ldg(p.rank_seg_ptr + r), e = __ldg(p.rank_seg_ptr + r + 1);
+      if (b >= 0 && b <= e && e <= p.rows) {
+        for (int j = b; j < e; ++j)
+          if (__ldg(p.rank_seg_idx + j) == s) {
+            // a rank buffer must be present, aligned to the vector type and
+            // long enough
+            const float *base = p.rank_G[r];
+            if (base != nullptr && (reinterpret_cast<uintptr_t>(base) % sizeof(V)) == 0 &&
+                j - b < p.rank_rows)
+              row = reinterpret_cast<const V *>(base) + (int64_t)(j - b) * p.cols;
+            break;
+          }
+      }
+    }
+    if (row == nullptr) ok = false;
+    s_rows[t] = row;
+  }
+  return ok;
+}
+
+template <typename V, bool kRanked>
 __global__ void __launch_bounds__(kThreads, MEP_REDUCE_MIN_BLOCKS) reduce_kernel(ReduceParams p) {
+  __shared__ const V *s_rows[kRanked ? kMaxSegPerExpert : 1];
   const V *G = reinterpret_cast<const V *>(p.G);
   V *home = reinterpret_cast<V *>(p.home);
   const int64_t tile = (int64_t)kThreads * kU;
   const int64_t tiles_per_e = (p.cols + tile - 1) / tile;
-  const int64_t ntask = (int64_t)p.E * tiles_per_e;
+  const int64_t ntask = (int64_t)p.ne * tiles_per_e;
   bool bad = false;
   for (int64_t task = blockIdx.x; task < ntask; task += gridDim.x) {
-    const int e = (int)(task / tiles_per_e);
-    const int64_t c0 = (task - (int64_t)e * tiles_per_e) * tile + threadIdx.x;
+    const int el = (int)(task / tiles_per_e);  // expert index within the reduced range
+    const int e = p.e0 + el;
+    const int64_t c0 = (task - (int64_t)el * tiles_per_e) * tile + threadIdx.x;
     int s0 = __ldg(p.eptr + e), s1 = __ldg(p.eptr + e + 1);
-    if (s0 < 0 || s1 < s0 || s1 > p.rows) {
+    if (s0 < 0 || s1 < s0 || s1 > p.rows || (kRanked && s1 - s0 > kMaxSegPerExpert)) {
       bad = true;
       s0 = s1 = 0;
+    }
+    if (kRanked) {
+      __syncthreads();  // the previous task's rows are no longer read
+      if (!resolve_rows<V>(p, s0, s1, s_rows)) bad = true;
+      __syncthreads();
     }
     V acc[kU];
 #pragma unroll
@@ -89,11 +154,11 @@ __global__ void __launch_bounds__(kThreads, MEP_REDUCE_MIN_BLOCKS) reduce_kernel
       V a[kSU][kU];
 #pragma unroll
       for (int q = 0; q < kSU; ++q) {
-        const V *row = G + (int64_t)(s + q) * p.cols;
+        const V *row = seg_row<V, kRanked>(p, G, s_rows, s + q, s0);
 #pragma unroll
         for (int j = 0; j < kU; ++j) {
           const int64_t c = c0 + (int64_t)j * kThreads;
-          if (c < p.cols) a[q][j] = __ldcs(row + c);
+          a[q][j] = (row != nullptr && c < p.cols) ? __ldcs(row + c) : zero_v<V>();
         }
       }
 #pragma unroll
@@ -103,18 +168,18 @@ __global__ void __launch_bounds__(kThreads, MEP_REDUCE_MIN_BLOCKS) reduce_kernel
           if (c0 + (int64_t)j * kThreads < p.cols) acc[j] = addv(acc[j], a[q][j]);
     }
     for (; s < s1; ++s) {
-      const V *row = G + (int64_t)s * p.cols;
+      const V *row = seg_row<V, kRanked>(p, G, s_rows, s, s0);
       V a[kU];
 #pragma unroll
       for (int j = 0; j < kU; ++j) {
         const int64_t c = c0 + (int64_t)j * kThreads;
-        if (c < p.cols) a[j] = __ldcs(row + c);
+        a[j] = (row != nullptr && c < p.cols) ? __ldcs(row + c) : zero_v<V>();
       }
 #pragma unroll
       for (int j = 0; j < kU; ++j)
         if (c0 + (int64_t)j * kThreads < p.cols) acc[j] = addv(acc[j], a[j]);
     }
-    V *hrow = home + (int64_t)e * p.cols;
+    V *hrow = home + (int64_t)el * p.cols;
 #pragma unroll
     for (int j = 0; j < kU; ++j) {
       const int64_t c = c0 + (int64_t)j * kThreads;
@@ -124,15 +189,31 @@ __global__ void __launch_bounds__(kThreads, MEP_REDUCE_MIN_BLOCKS) reduce_kernel
   if (bad) set_status(p.status, MEP_ERR_DEVICE_DATA);
 }
 
-}  // namespace
-
-cudaError_t launch_reduce(const mep_shape_t &s, const mep_plan_t &pl, int64_t P,
-                          const float *G, float *home, cudaStream_t stream) {
+template <bool kRanked>
+cudaError_t launch(ReduceParams &p, int64_t P, cudaStream_t stream) {
   int dev = 0, sms = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
   if ((err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
     return err;
+  const bool vec = (P % 4) == 0;
+  p.cols = vec ? P / 4 : P;
+  const int64_t tile = (int64_t)kThreads * kU;
+  const int64_t ntask = (int64_t)p.ne * ((p.cols + tile - 1) / tile);
+  if (ntask == 0) return cudaSuccess;
+  const int blocks =
+      (int)std::max<int64_t>(1, std::min<int64_t>(ntask, (int64_t)sms * MEP_REDUCE_BLOCKS_PER_SM));
+  if (vec)
+    reduce_kernel<float4, kRanked><<<blocks, kThreads, 0, stream>>>(p);
+  else
+    reduce_kernel<float, kRanked><<<blocks, kThreads, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_reduce(const mep_shape_t &s, const mep_plan_t &pl, int64_t P,
+                          const float *G, float *home, cudaStream_t stream) {
   ReduceParams p{};
   p.G = G;
   p.home = home;
@@ -140,17 +221,30 @@ cudaError_t launch_reduce(const mep_shape_t &s, const mep_plan_t &pl, int64_t P,
   p.status = pl.status;
   p.E = s.E;
   p.rows = s.E + s.R - 1;
-  const bool vec = (P % 4) == 0;
-  p.cols = vec ? P / 4 : P;
-  const int64_t tile = (int64_t)kThreads * kU;
-  const int64_t ntask = (int64_t)s.E * ((p.cols + tile - 1) / tile);
-  const int blocks =
-      (int)std::max<int64_t>(1, std::min<int64_t>(ntask, (int64_t)sms * MEP_REDUCE_BLOCKS_PER_SM));
-  if (vec)
-    reduce_kernel<float4><<<blocks, kThreads, 0, stream>>>(p);
-  else
-    reduce_kernel<float><<<blocks, kThreads, 0, stream>>>(p);
-  return cudaGetLastError();
+  p.R = s.R;
+  p.e0 = 0;
+  p.ne = s.E;
+  return launch<false>(p, P, stream);
+}
+
+cudaError_t launch_reduce_ranked(const mep_shape_t &s, const mep_plan_t &pl, int64_t P,
+                                 int32_t home_rank, const float *const *rank_G,
+                                 int64_t rank_rows, float *home, cudaStream_t stream) {
+  ReduceParams p{};
+  p.home = home;
+  p.eptr = pl.expert_seg_ptr;
+  p.status = pl.status;
+  p.E = s.E;
+  p.rows = s.E + s.R - 1;
+  p.rank_G = rank_G;
+  p.rank_rows = rank_rows;
+  p.seg = reinterpret_cast<const int4 *>(pl.seg);
+  p.rank_seg_ptr = pl.rank_seg_ptr;
+  p.rank_seg_idx = pl.rank_seg_idx;
+  p.R = s.R;
+  p.ne = s.E / s.R;
+  p.e0 = home_rank * p.ne;
+  return launch<true>(p, P, stream);
 }
 
 }  // namespace mep
