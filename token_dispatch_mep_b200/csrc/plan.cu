@@ -272,7 +272,10 @@ __global__ void __launch_bounds__(kThreads, 1) plan_kernel(PlanParams p) {
   if (!plan_sync(p, 2)) return;
 
   // ---- phase 3: offsets, scalars, segments, scatter -------------------------
+  // Both loads issued together: one L2 round trip before the scans.
   const int T = t < E ? __ldcg(p.counts + t) : 0;
+  const int tile_off =
+      (p.full && !coord && t < E) ? __ldcg(p.tile + (int64_t)t * p.nt + tile) : 0;
   int total;
   const int off = block_excl_scan(T, &total, s_w);
   if (t < E) s_off[t] = off;
@@ -461,7 +464,7 @@ __global__ void __launch_bounds__(kThreads, 1) plan_kernel(PlanParams p) {
   if (p.full && !coord) {
     // Per-warp cursors: expert offset + tile offset + warp offset.
     if (t < E) {
-      const int base = off + __ldcg(p.tile + (int64_t)t * p.nt + tile);
+      const int base = off + tile_off;
       for (int w = 0; w < kWarps; ++w) wh_all[w * E + t] += base;
     }
     __syncthreads();
