@@ -19,7 +19,10 @@
 // 0.90-1.00 of the HBM copy peak against 0.96-1.04 for this one.
 //
 // Rank-addressed form (mep_combine_ranked): expert outputs are read from R
-// separate rank buffers, slot p being row p % SK of rank_ys[p / SK].
+// separate rank buffers, slot p being row p % SK of rank_ys[p / SK]; a NULL
+// or misaligned rank pointer is reported, never used.  A token range [g0, g0
+// + N) restricts the kernel to one rank's own tokens (out and w rows are the
+// range's; mep_combine_ranked_tokens).
 //
 // With no weights (w == nullptr) every weight is 1 and the kernel is the
 // backward of dispatch: grad_x[g] = bf16(sum_k grad_buf[slot[g,k]]) (an FMA

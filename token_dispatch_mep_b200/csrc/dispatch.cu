@@ -26,11 +26,14 @@
 // Rank-addressed form (mep_dispatch_ranked): rank r's S*K slots live in
 // their own buffer rank_bufs[r] (on a multi-GPU system a peer buffer mapped
 // into this GPU's address space), so slot p is row p % SK of rank_bufs[p / SK]
-// and each store goes straight to the rank that owns the slot.
+// and each store goes straight to the rank that owns the slot; a NULL or
+// misaligned rank pointer is reported, never used.  A token range [g0, g0 +
+// N) restricts the kernel to one rank's own tokens (mep_dispatch_ranked_tokens).
 //
 // A bulk-copy (TMA) design -- rows staged in shared memory by bulk loads on
 // mbarriers, K bulk stores per row -- measured 0.82-0.87 of the HBM copy
-// peak on this path against 0.89-0.94 for this one, so it is not used.
+// peak on this path against 0.89-0.94 for the register path at the time
+// (0.99-1.03 now), so it is not used.
 #include <algorithm>
 #include <atomic>
 #include <cstdint>
