@@ -106,7 +106,14 @@ def _case_gather_ids(rank, world):
                         starts == sorted(starts) and (not starts or starts[0] == 0),
                         len(segs) <= ep.max_local_segments(type("Sh", (), dict(E=E, SK=S * K))()),
                         len(set(experts)) == len(experts)))
-    return same, covered
+    errors = []
+    for shape, sched in (((3, 4, 6, 2), "contiguous"), ((2, 4, 6, 2), "fastest")):
+        try:
+            ep.ExchangeGroup(shape, 8, 0, device="cpu", schedule=sched)
+            errors.append(None)
+        except ValueError as e:           # rejected before any buffer is made
+            errors.append(type(e).__name__)
+    return same, covered, errors
 
 
 CASES = {"max": _case_max, "sharded_plan": _case_sharded_plan, "gather_ids": _case_gather_ids}
@@ -156,7 +163,8 @@ def test_reference_arm_prints_on_rank_zero_only(monkeypatch):
 def test_router_id_gather_and_local_segment_lists():
     out = _run("gather_ids")
     for rank in (0, 1):
-        same, covered = out[rank]
+        same, covered, errors = out[rank]
         assert same is True, out
         for flags in covered:                   # contiguous, home-first
             assert all(flags), (rank, flags)
+        assert errors == ["ValueError", "ValueError"], errors  # R != world size; unknown schedule
