@@ -33,6 +33,10 @@
 //            offset + rank among equal ids earlier in the warp.  The rank
 //            comes from a peer mask (one ballot per id bit; the lanes holding
 //            the same id) and the popcount of the peers below the lane.
+//            The per-pair work of this loop is what bounds phase 3 on large
+//            workloads (the SM's instruction issue, measured ~0.9 us per
+//            32-pair step of the 32 warps); staging src_pair through shared
+//            memory to coalesce its scattered stores was measured slower.
 // A warp whose range exceeds its shared-memory id buffer reads its ids again
 // from global memory (L2 hits) in phase 3.
 #include <atomic>
@@ -189,23 +193,26 @@ __global__ void __launch_bounds__(kThreads, 1) plan_kernel(PlanParams p) {
   const int64_t w0 = b0 + (n * warp) / kWarps;
   const int64_t w1 = b0 + (n * (warp + 1)) / kWarps;
   const bool keep = (w1 - w0) <= kPlanIdsPerWarp;  // ids stay in shared memory
+  // 32-bit indices inside the warp's range (NK < 2^31 by the shape rules).
+  const int nw = (int)(w1 - w0);
+  const int32_t *idx_w = p.idx + w0;
 
   // ---- phase 1: warp-private histograms ------------------------------------
   bool bad = false;
-  for (int64_t c = w0; c < w1; c += 32 * kBatch) {
+  for (int c = 0; c < nw; c += 32 * kBatch) {
     int ev[kBatch];
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
-      const int64_t q = c + u * 32 + lane;
-      ev[u] = q < w1 ? __ldg(p.idx + q) : -1;
+      const int i = c + u * 32 + lane;
+      ev[u] = i < nw ? __ldg(idx_w + i) : -1;
     }
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
-      const int64_t q = c + u * 32 + lane;
-      if (q < w1) {
+      const int i = c + u * 32 + lane;
+      if (i < nw) {
         const int e = ev[u];
         if ((unsigned)e < (unsigned)E) atomicAdd(wh + e, 1); else bad = true;
-        if (keep) ids[q - w0] = e;
+        if (keep) ids[i] = e;
       }
     }
   }
@@ -462,32 +469,36 @@ __global__ void __launch_bounds__(kThreads, 1) plan_kernel(PlanParams p) {
   }
 
   if (p.full && !coord) {
-    // Per-warp cursors: expert offset + tile offset + warp offset.
-    if (t < E) {
-      const int base = off + tile_off;
-      for (int w = 0; w < kWarps; ++w) wh_all[w * E + t] += base;
-    }
+    // Per expert: where this tile's pairs start in the expert-sorted order
+    // (expert offset + tile offset); wh keeps the warp offsets in the tile.
+    int *s_base = s_tab[7];
+    __syncthreads();  // a single block has finished the coordinator's tables
+    if (t < E) s_base[t] = off + tile_off;
     __syncthreads();
 
     const bool hf = p.kind == kPlanHomeFirst;
     const unsigned lt = lanemask_lt();
-    for (int64_t c = w0; c < w1; c += 32) {
-      const int64_t q = c + lane;
-      const bool act = q < w1;
+    const unsigned nk = (unsigned)p.NK;
+    int32_t *slot_w = p.slot + w0;
+    const int q0 = (int)w0;
+    for (int c = 0; c < nw; c += 32) {
+      const int i = c + lane;
+      const bool act = i < nw;
       int e = -1;
-      if (act) e = keep ? ids[q - w0] : __ldg(p.idx + q);
+      if (act) e = keep ? ids[i] : __ldg(idx_w + i);
       const bool valid = (unsigned)e < (unsigned)E;
       const unsigned peers = peers_of(valid ? e : sentinel, nbits);
-      const int base = valid ? wh[e] : 0;
+      const int wo = valid ? wh[e] : 0;
       __syncwarp();
       if (valid) {
-        int s = base + __popc(peers & lt);  // position in the expert-sorted order
+        const int r = wo + __popc(peers & lt);  // rank among the tile's pairs of e
+        int s = s_base[e] + r;                  // position in the expert-sorted order
         if (hf) s = home_first_slot(e, s - s_off[e], Bx, C, p.R, s_h, s_off, s_O, s_F, s_D);
-        p.slot[q] = s;
-        if ((unsigned)s < (unsigned)p.NK) p.src_pair[s] = (int32_t)q;
-        if (lane == __ffs(peers) - 1) wh[e] = base + __popc(peers);
+        slot_w[i] = s;
+        if ((unsigned)s < nk) p.src_pair[s] = q0 + i;
+        if (lane == __ffs(peers) - 1) wh[e] = wo + __popc(peers);
       } else if (act) {
-        p.slot[q] = -1;
+        slot_w[i] = -1;
       }
       __syncwarp();
     }
