@@ -3,9 +3,9 @@ process group for the host-side exchange), their buffers shared by CUDA IPC
 handles, each rank dispatching, combining and reducing its own share through
 the peer mappings (``token_dispatch_mep_b200.ep``).
 
-This pool gives one GPU per run, so both processes use cuda:0 -- which CUDA
-IPC supports -- and the ranks are ordered by host barriers only: no kernel
-of one rank waits on a kernel of the other.  Every rank checks its own
+The test needs only one GPU: both processes use cuda:0 -- which CUDA IPC
+supports -- and the ranks are ordered by host barriers only: no kernel of
+one rank waits on a kernel of the other.  Every rank checks its own
 receive buffer, combine output and home-expert gradients against the oracle
 (bit-exact dispatch; combine within 1 bf16 ulp; reduce within the fp32
 bound)."""
