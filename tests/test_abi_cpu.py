@@ -171,3 +171,11 @@ def test_host_side_rejections_of_the_exchange_calls(lib):
     assert L.mep_ipc_open(ctypes.byref(h), None) == 1
     assert L.mep_ipc_close(None, good) == 1
     assert L.mep_ipc_close(ctypes.byref(h), None) == 1
+
+
+def test_python_modules_import_without_a_gpu():
+    """The autograd wrappers and the exchange module load on a CPU-only host;
+    their work happens only when called on CUDA tensors."""
+    from token_dispatch_mep_b200 import autograd, ep
+    assert callable(autograd.dispatch) and callable(autograd.combine)
+    assert callable(ep.gather_router_ids) and ep.max_local_segments(mep.Shape(8, 4096, 64, 6)) == 64
