@@ -26,6 +26,10 @@
 //   Phase 2  one warp per expert scans its row tile[e][0..nt) into exclusive
 //            per-tile offsets and writes T_e.
 //   -- grid barrier --
+//            When the tile matrix is small (at most 8 entries per thread)
+//            every block instead reads all of it and sums T_e and its own
+//            tile offsets itself: no second grid barrier, no write-back of
+//            the matrix.
 //   Phase 3  every block scans T_e over experts (expert offsets); the
 //            coordinator writes maxvio, the offsets, segments, CSR pointers
 //            and replica list; every tile warp walks its ids again in (g, k)
@@ -55,6 +59,7 @@ constexpr int kThreads = kPlanThreads;
 constexpr int kWarps = kThreads / 32;
 constexpr int kBatch = 8;          // 32-pair chunks a warp loads at once
 constexpr int kTab = MEP_MAX_EXPERTS + 1;
+constexpr int kDirectLoads = 8;  // tile-matrix entries per thread in the direct phase 2
 
 #ifndef MEP_PLAN_PEERS_BALLOT
 #define MEP_PLAN_PEERS_BALLOT 1  // 1: peer masks from bit ballots; 0: match.any
@@ -232,7 +237,35 @@ __global__ void __launch_bounds__(kThreads, 1) plan_kernel(PlanParams p) {
   if (bad && t == 0) set_status(p.status, MEP_ERR_DEVICE_DATA);
 
   // ---- phase 2: per-expert scan over tiles ----------------------------------
-  {
+  int tpe = 32;  // direct form: threads per expert, a power of two (groups inside a warp)
+  while (tpe > 1 && tpe * E > kThreads) tpe >>= 1;
+  const bool direct = p.nb > 1 && p.nt <= kDirectLoads * tpe;
+  int *s_T = s_tab[5], *s_pre = s_tab[6];  // direct form: T_e, this tile's offsets
+  if (direct) {
+    const int e = t / tpe, sub = t % tpe;
+    const int32_t *row = p.tile + (int64_t)min(e, E - 1) * p.nt;
+    int v[kDirectLoads];
+#pragma unroll
+    for (int j = 0; j < kDirectLoads; ++j) {  // all loads in flight together
+      const int b = sub + j * tpe;
+      v[j] = (e < E && b < p.nt) ? __ldcg(row + b) : 0;
+    }
+    int tot = 0, pre = 0;
+#pragma unroll
+    for (int j = 0; j < kDirectLoads; ++j) {
+      tot += v[j];
+      if (sub + j * tpe < tile) pre += v[j];
+    }
+    for (int o = tpe >> 1; o > 0; o >>= 1) {
+      tot += __shfl_xor_sync(0xffffffffu, tot, o);
+      pre += __shfl_xor_sync(0xffffffffu, pre, o);
+    }
+    if (e < E && sub == 0) {
+      s_T[e] = tot;
+      s_pre[e] = pre;
+    }
+    __syncthreads();
+  } else {
     const int per = (p.nt + 31) / 32;  // tiles per lane, <= 32
     for (int e = blockIdx.x * kWarps + warp; e < E; e += p.nb * kWarps) {
       int32_t *row = p.tile + (int64_t)e * p.nt;
@@ -276,13 +309,16 @@ __global__ void __launch_bounds__(kThreads, 1) plan_kernel(PlanParams p) {
     }
   }
 
-  if (!plan_sync(p, 2)) return;
+  if (!direct && !plan_sync(p, 2)) return;
 
   // ---- phase 3: offsets, scalars, segments, scatter -------------------------
   // Both loads issued together: one L2 round trip before the scans.
-  const int T = t < E ? __ldcg(p.counts + t) : 0;
+  const int T = t < E ? (direct ? s_T[t] : __ldcg(p.counts + t)) : 0;
   const int tile_off =
-      (p.full && !coord && t < E) ? __ldcg(p.tile + (int64_t)t * p.nt + tile) : 0;
+      (p.full && !coord && t < E)
+          ? (direct ? s_pre[t] : __ldcg(p.tile + (int64_t)t * p.nt + tile))
+          : 0;
+  if (direct && blockIdx.x == 0 && t < E) p.counts[t] = T;
   int total;
   const int off = block_excl_scan(T, &total, s_w);
   if (t < E) s_off[t] = off;
@@ -313,10 +349,15 @@ __global__ void __launch_bounds__(kThreads, 1) plan_kernel(PlanParams p) {
       pre = min(before, C);
       over = T - h;
     }
-    int otot, hptot, optot;
+    int otot, hptot = 0, optot = 0;
     const int O = block_excl_scan(over, &otot, s_w);
-    const int hp = block_excl_scan(h > 0 ? 1 : 0, &hptot, s_w);
-    const int op = block_excl_scan(over > 0 ? 1 : 0, &optot, s_w);
+    // The piece counts before each expert are only needed for the
+    // coordinator's tables.
+    int hp = 0, op = 0;
+    if (blockIdx.x == 0) {
+      hp = block_excl_scan(h > 0 ? 1 : 0, &hptot, s_w);
+      op = block_excl_scan(over > 0 ? 1 : 0, &optot, s_w);
+    }
     int F = 0, room = 0;
     if (t < p.R) {
       const int load = s_off[(t + 1) * Bx] - s_off[t * Bx];
