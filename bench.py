@@ -362,6 +362,8 @@ def main():
     value = whole_job_rate(N, world, ms_step)
 
     stage_ms = dict(zip(["plan", "dispatch", "combine", "reduce"], stage.mean(axis=0).tolist()))
+    # plan + dispatch + combine alone (the rate the metric names), slowest rank
+    pdc_ms = max_over_ranks(stage_ms["plan"] + stage_ms["dispatch"] + stage_ms["combine"], world, dev)
     algo = {
         "plan": 3 * NK * 4,
         "dispatch": N * H * 2 + NK * H * 2 + NK * 4,
@@ -560,7 +562,6 @@ def main():
     if graph is not None:   # headline: the step as a user runs it, one graph replay per step
         ms_step, value = graph["ms_per_step"], graph["value"]
     if rank == 0:
-        pdc_ms = stage_ms["plan"] + stage_ms["dispatch"] + stage_ms["combine"]
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
