@@ -151,14 +151,18 @@ __device__ __forceinline__ int upper_bound_idx(const int *a, int n, int x) {
 }
 
 // Slot of the i-th pair (in (g,k) order) of expert e in the home-first plan.
+// s_rf[e] is the first rank of e's overflow; the pair's rank, the first r
+// with D[r+1] > q, is found by stepping from there (an expert's overflow
+// spans few ranks).
 __device__ __forceinline__ int home_first_slot(int e, int i, int Bx, int C, int R, const int *s_h,
                                                const int *s_off, const int *s_O, const int *s_F,
-                                               const int *s_D) {
+                                               const int *s_D, const int *s_rf) {
   const int h = s_h[e];
   const int home = e / Bx;
   if (i < h) return home * C + (s_off[e] - s_off[home * Bx]) + i;
   const int q = s_O[e] + (i - h);
-  const int r = upper_bound_idx(s_D + 1, R, q);  // first rank with D[r+1] > q
+  int r = s_rf[e];
+  while (r < R - 1 && s_D[r + 1] <= q) ++r;
   return r * C + s_F[r] + (q - s_D[r]);
 }
 
@@ -175,6 +179,8 @@ __global__ void __launch_bounds__(kThreads, 1) plan_kernel(PlanParams p) {
   __shared__ int s_w[32];
   // Tables over experts (or ranks), E + 1 <= kTab entries each.
   __shared__ int s_tab[8][kTab];
+  __shared__ int s_rank[MEP_MAX_RANKS];  // home-first coordinator: per-rank index base
+  __shared__ int s_rf[MEP_MAX_EXPERTS];  // home-first: first rank of each expert's overflow
   int *s_off = s_tab[0];   // expert offsets (exclusive prefix of T_e), [E] = total
 
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
@@ -354,9 +360,13 @@ __global__ void __launch_bounds__(kThreads, 1) plan_kernel(PlanParams p) {
     // The piece counts before each expert are only needed for the
     // coordinator's tables.
     int hp = 0, op = 0;
-    if (blockIdx.x == 0) {
-      hp = block_excl_scan(h > 0 ? 1 : 0, &hptot, s_w);
-      op = block_excl_scan(over > 0 ? 1 : 0, &optot, s_w);
+    if (blockIdx.x == 0) {  // both counts (<= E < 2^16) in one scan
+      int both_tot;
+      const int both = block_excl_scan((h > 0 ? 1 : 0) | ((over > 0 ? 1 : 0) << 16), &both_tot, s_w);
+      hp = both & 0xffff;
+      op = both >> 16;
+      hptot = both_tot & 0xffff;
+      optot = both_tot >> 16;
     }
     int F = 0, room = 0;
     if (t < p.R) {
@@ -383,33 +393,37 @@ __global__ void __launch_bounds__(kThreads, 1) plan_kernel(PlanParams p) {
       s_D[p.R] = dtot;
     }
     __syncthreads();
+    if (t < E) s_rf[t] = over > 0 ? upper_bound_idx(s_D + 1, p.R, O) : 0;
+    __syncthreads();
   }
 
   if (p.full && blockIdx.x == 0) {  // the coordinator (or the only block)
     if (p.kind == kPlanContiguous) {
-      const int64_t SK = p.SK;
+      // Slot positions are < N*K < 2^31: 32-bit arithmetic throughout.
+      const int SK = (int)p.SK;
       int *s_sbase = s_tab[1];
       int nseg_e = 0, r0 = 0, r1 = -1;
       if (t < E && T > 0) {
-        r0 = (int)(off / SK);
-        r1 = (int)((off + (int64_t)T - 1) / SK);
+        r0 = (int)((unsigned)off / (unsigned)SK);
+        r1 = (int)((unsigned)(off + T - 1) / (unsigned)SK);
         nseg_e = r1 - r0 + 1;
       }
-      int nseg;
-      const int sbase = block_excl_scan(nseg_e, &nseg, s_w);
       const int home = t / Bx;
       const int nrep_e = nseg_e - ((nseg_e > 0 && home >= r0 && home <= r1) ? 1 : 0);
-      int nrep;
-      int rbase = block_excl_scan(nrep_e, &nrep, s_w);
+      // segment and replica counts (totals <= E + R - 1 < 2^16) in one scan
+      int both_tot;
+      const int both = block_excl_scan(nseg_e | (nrep_e << 16), &both_tot, s_w);
+      const int sbase = both & 0xffff, nseg = both_tot & 0xffff, nrep = both_tot >> 16;
+      int rbase = both >> 16;
       if (t < E) {
         s_sbase[t] = sbase;
         p.expert_offset[t] = off;
         p.expert_seg_ptr[t] = sbase;
         for (int j = 0; j < nseg_e; ++j) {
           const int r = r0 + j;
-          const int64_t lo = max((int64_t)off, (int64_t)r * SK);
-          const int64_t hi = min((int64_t)off + T, (int64_t)(r + 1) * SK);
-          p.seg[sbase + j] = make_int4(t, r, (int)(lo - (int64_t)r * SK), (int)(hi - lo));
+          const int lo = max(off, r * SK);
+          const int hi = min(off + T, (r + 1) * SK);
+          p.seg[sbase + j] = make_int4(t, r, lo - r * SK, hi - lo);
           p.rank_seg_idx[sbase + j] = sbase + j;  // slot order is table order
           if (r != home) p.replica_seg[rbase++] = sbase + j;
         }
@@ -423,16 +437,10 @@ __global__ void __launch_bounds__(kThreads, 1) plan_kernel(PlanParams p) {
       }
       __syncthreads();
       for (int r = t; r <= p.R; r += kThreads) {
-        const int64_t x = (int64_t)r * SK;
         int ptr = nseg;
-        if (r < p.R && x < total) {
-          int lo = 0, hi = E + 1;  // first index with s_off > x
-          while (lo < hi) {
-            const int mid = (lo + hi) >> 1;
-            if ((int64_t)s_off[mid] <= x) lo = mid + 1; else hi = mid;
-          }
-          const int e = lo - 1;
-          ptr = s_sbase[e] + (r - (int)(s_off[e] / SK));
+        if (r < p.R && r * SK < total) {
+          const int e = upper_bound_idx(s_off, E + 1, r * SK) - 1;  // expert holding slot r*SK
+          ptr = s_sbase[e] + (r - (int)((unsigned)s_off[e] / (unsigned)SK));
         }
         p.rank_seg_ptr[r] = ptr;
       }
@@ -441,12 +449,12 @@ __global__ void __launch_bounds__(kThreads, 1) plan_kernel(PlanParams p) {
       const int R = p.R;
       // Per rank: home pieces (home experts keeping pairs) + replica pieces
       // (overflowing experts whose overflow meets the rank's spare room).
-      int nh = 0, nr = 0;
+      int nh = 0, nr = 0, ef = 0;
       if (t < R) {
         nh = s_hp[(t + 1) * Bx] - s_hp[t * Bx];
         const int d0 = s_D[t], d1 = s_D[t + 1];
         if (d1 > d0) {
-          const int ef = upper_bound_idx(s_O, E + 1, d0) - 1;       // expert holding d0
+          ef = upper_bound_idx(s_O, E + 1, d0) - 1;                 // expert holding d0
           const int el = upper_bound_idx(s_O, E + 1, d1 - 1) - 1;   // expert holding d1 - 1
           nr = s_op[el + 1] - s_op[ef];
         }
@@ -455,6 +463,9 @@ __global__ void __launch_bounds__(kThreads, 1) plan_kernel(PlanParams p) {
       const int rsp = block_excl_scan(nh + nr, &ntot, s_w);
       if (t < R) {
         s_rsp[t] = rsp;
+        // rank t's replica piece of an overflowing expert e sits at
+        // s_rank[t] + s_op[e] in its list (after its nh home pieces)
+        s_rank[t] = rsp + nh - s_op[ef];
         p.rank_seg_ptr[t] = rsp;
       }
       if (t == 0) {
@@ -467,16 +478,19 @@ __global__ void __launch_bounds__(kThreads, 1) plan_kernel(PlanParams p) {
       int rf = 0, rl = -1;
       if (t < E && over > 0) {
         const int O = s_O[t];
-        rf = upper_bound_idx(s_D + 1, R, O);                 // first rank with D[r+1] > O
+        rf = s_rf[t];                                        // first rank with D[r+1] > O
         rl = upper_bound_idx(s_D + 1, R, O + over - 1);      // rank holding the last pair
       }
       int nrep_e = 0;
       for (int r = rf; r <= rl; ++r)
         if (s_D[r + 1] > s_D[r]) ++nrep_e;
       const int nseg_e = nrep_e + (h > 0 ? 1 : 0);
-      int nseg, nrep;
-      int sidx = block_excl_scan(nseg_e, &nseg, s_w);
-      int ridx = block_excl_scan(nrep_e, &nrep, s_w);
+      // segment and replica counts (totals <= E + R - 1 < 2^16) in one scan
+      int both_tot;
+      const int both = block_excl_scan(nseg_e | (nrep_e << 16), &both_tot, s_w);
+      const int nseg = both_tot & 0xffff, nrep = both_tot >> 16;
+      int sidx = both & 0xffff;
+      int ridx = both >> 16;
       if (t < E) {
         const int home = t / Bx;
         p.expert_offset[t] = off;
@@ -493,9 +507,7 @@ __global__ void __launch_bounds__(kThreads, 1) plan_kernel(PlanParams p) {
           if (r > rl || s_D[r + 1] <= s_D[r]) continue;
           const int lo = max(O, s_D[r]), hi = min(O + over, s_D[r + 1]);
           p.seg[sidx] = make_int4(t, r, s_F[r] + (lo - s_D[r]), hi - lo);
-          const int ef = upper_bound_idx(s_O, E + 1, s_D[r]) - 1;
-          const int nh_r = s_hp[(r + 1) * Bx] - s_hp[r * Bx];
-          p.rank_seg_idx[s_rsp[r] + nh_r + (s_op[t] - s_op[ef])] = sidx;
+          p.rank_seg_idx[s_rank[r] + s_op[t]] = sidx;
           p.replica_seg[ridx++] = sidx;
           ++sidx;
         }
@@ -534,7 +546,7 @@ __global__ void __launch_bounds__(kThreads, 1) plan_kernel(PlanParams p) {
       if (valid) {
         const int r = wo + __popc(peers & lt);  // rank among the tile's pairs of e
         int s = s_base[e] + r;                  // position in the expert-sorted order
-        if (hf) s = home_first_slot(e, s - s_off[e], Bx, C, p.R, s_h, s_off, s_O, s_F, s_D);
+        if (hf) s = home_first_slot(e, s - s_off[e], Bx, C, p.R, s_h, s_off, s_O, s_F, s_D, s_rf);
         slot_w[i] = s;
         if ((unsigned)s < nk) p.src_pair[s] = q0 + i;
         if (lane == __ffs(peers) - 1) wh[e] = wo + __popc(peers);
