@@ -179,3 +179,23 @@ def test_python_modules_import_without_a_gpu():
     from token_dispatch_mep_b200 import autograd, ep
     assert callable(autograd.dispatch) and callable(autograd.combine)
     assert callable(ep.gather_router_ids) and ep.max_local_segments(mep.Shape(8, 4096, 64, 6)) == 64
+
+
+def test_rank_pointer_table_keeps_its_buffers_alive():
+    """A table made from temporary rank buffers must not outlive them: the
+    table holds references, so the addresses it carries stay allocated."""
+    import gc
+    import weakref
+
+    import torch
+    s = mep.Shape(2, 3, 4, 2)
+    H = 8
+    table = mep.rank_pointer_table([torch.zeros((s.SK, H), dtype=torch.bfloat16) for _ in range(2)],
+                                   s, H, "cpu")
+    refs = [weakref.ref(b) for b in table.keepalive]
+    gc.collect()
+    assert all(r() is not None for r in refs)
+    assert table.tolist() == [b.data_ptr() for b in table.keepalive]
+    del table
+    gc.collect()
+    assert all(r() is None for r in refs)

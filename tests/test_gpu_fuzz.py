@@ -1,0 +1,99 @@
+"""Randomised parity (hypothesis, derandomised): small random shapes and
+routings -- skewed, duplicate ids inside a token, everything on one expert,
+ids at the edges of [0, E) -- through the C ABI on the GPU, against the
+oracle: both plans bit-exact, dispatch bit-exact, combine and reduce within
+the contract's tolerances, and one rank's token range of the rank-addressed
+calls equal to the whole-range result."""
+import numpy as np
+import pytest
+import torch
+from hypothesis import HealthCheck, given, settings
+from hypothesis import strategies as st
+
+import oracle
+import parity
+import token_dispatch_mep_b200 as mep
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+SETTINGS = settings(max_examples=60, deadline=None, derandomize=True,
+                    suppress_health_check=[HealthCheck.too_slow, HealthCheck.function_scoped_fixture])
+
+
+def _u16(t):
+    return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+@st.composite
+def case(draw):
+    R = draw(st.integers(1, 8))
+    B = draw(st.integers(1, 6))
+    E = R * B
+    K = draw(st.integers(1, min(E, 16)))
+    S = draw(st.integers(1, 90))
+    H = 8 * draw(st.integers(1, 40))
+    P = draw(st.integers(1, 70))
+    kind = draw(st.sampled_from(["distinct", "dups", "one", "skew", "edges"]))
+    seed = draw(st.integers(0, 2 ** 31 - 1))
+    rng = np.random.default_rng(seed)
+    N = R * S
+    if kind == "distinct":
+        idx = np.argsort(-rng.standard_normal((N, E)), axis=1, kind="stable")[:, :K]
+    elif kind == "skew":
+        logits = rng.standard_normal((N, E)) - 3.0 * np.log(np.arange(1, E + 1))
+        idx = np.argsort(-logits, axis=1, kind="stable")[:, :K]
+    elif kind == "dups":
+        idx = rng.integers(0, E, size=(N, K))
+    elif kind == "edges":
+        idx = rng.choice(np.array([0, E - 1]), size=(N, K))
+    else:
+        idx = np.full((N, K), int(rng.integers(0, E)))
+    w = rng.standard_normal((N, K)).astype(np.float32)
+    return R, S, E, K, H, P, np.ascontiguousarray(idx, dtype=np.int32), w, seed
+
+
+@SETTINGS
+@given(case())
+def test_random_shapes_against_the_oracle(c):
+    R, S, E, K, H, P, idx, w, seed = c
+    ora = oracle.get()
+    N, NK, SK = R * S, R * S * K, S * K
+    s = mep.Shape(R, S, E, K)
+    gen = torch.Generator().manual_seed(seed)
+    x = torch.randn((N, H), generator=gen).to(torch.bfloat16)
+    y = torch.randn((NK, H), generator=gen).to(torch.bfloat16)
+    G = torch.randn((E + R - 1, P), generator=gen)
+    for home_first in (False, True):
+        plan = mep.Plan(s, DEV)
+        (mep.mep_plan_home_first if home_first else mep.mep_plan)(s, torch.from_numpy(idx).to(DEV), plan)
+        pl = (ora.plan_home_first if home_first else ora.plan)(R, S, E, K, idx)
+        buf = torch.empty((NK, H), dtype=torch.bfloat16, device=DEV)
+        out = torch.empty((N, H), dtype=torch.bfloat16, device=DEV)
+        home = torch.empty((E, P), dtype=torch.float32, device=DEV)
+        mep.mep_dispatch(s, H, plan, x.to(DEV), buf)
+        mep.mep_combine(s, H, plan, y.to(DEV), torch.from_numpy(w).to(DEV), out)
+        mep.mep_reduce_replica_grads(s, plan, P, G.to(DEV), home)
+        # one rank's share through the rank-addressed per-rank calls
+        r = int(seed % R)
+        bufs = [torch.full((SK, H), -1, dtype=torch.int16, device=DEV).view(torch.bfloat16)
+                for _ in range(R)]
+        mep.mep_dispatch_ranked_tokens(s, H, plan, r * S, x[r * S:(r + 1) * S].to(DEV),
+                                       mep.rank_pointer_table(bufs, s, H, DEV))
+        out_r = torch.empty((S, H), dtype=torch.bfloat16, device=DEV)
+        ys = [y[q * SK:(q + 1) * SK].to(DEV) for q in range(R)]
+        ytab = mep.rank_pointer_table(ys, s, H, DEV)
+        mep.mep_combine_ranked_tokens(s, H, plan, r * S, ytab,
+                                      torch.from_numpy(w[r * S:(r + 1) * S].copy()).to(DEV), out_r)
+        assert mep.mep_read_status(plan) == 0
+        parity.check_plan(plan.host(), pl, f"fuzz hf={home_first}")
+        assert np.array_equal(_u16(buf), ora.dispatch(K, pl["src_pair"], _u16(x)))
+        ob, ex, ab = ora.combine(pl["slot"], w, _u16(y))
+        parity.check_combine(_u16(out), ob, ex, ab, K, "fuzz")
+        hexact, habs = ora.reduce(pl["expert_seg_ptr"], G.numpy())
+        parity.check_reduce(home.cpu().numpy(), hexact, habs, np.diff(pl["expert_seg_ptr"]), "fuzz")
+        assert torch.equal(out_r.view(torch.int16), out[r * S:(r + 1) * S].view(torch.int16))
+        mine = np.unique(pl["slot"][r * S:(r + 1) * S].reshape(-1))
+        flat = torch.cat(bufs)
+        assert torch.equal(flat[torch.from_numpy(mine).to(DEV).long()].view(torch.int16),
+                           buf[torch.from_numpy(mine).to(DEV).long()].view(torch.int16))

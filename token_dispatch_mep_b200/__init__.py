@@ -338,13 +338,18 @@ def mep_prefetch_replica_weights(shape, plan: Plan, w_home, w_rep):
 
 
 def rank_pointer_table(bufs, shape, H: int, device) -> torch.Tensor:
-    """Device array of the R rank buffers' addresses (each [S*K, H] bf16)."""
+    """Device array of the R rank buffers' addresses (each [S*K, H] bf16).
+    The returned table holds references to the buffers, so they stay
+    allocated for as long as the table is alive."""
     s = _shape(shape)
+    bufs = list(bufs)
     if len(bufs) != s.R:
         raise ValueError(f"{len(bufs)} rank buffers, need {s.R}")
     for r, b in enumerate(bufs):
         _need(b, f"rank buffer {r}", torch.bfloat16, s.SK * H, torch.device(device))
-    return torch.tensor([b.data_ptr() for b in bufs], dtype=torch.int64, device=device)
+    table = torch.tensor([b.data_ptr() for b in bufs], dtype=torch.int64, device=device)
+    table.keepalive = bufs
+    return table
 
 
 def mep_dispatch_ranked(shape, H: int, plan: Plan, x, rank_table):
@@ -371,7 +376,8 @@ def mep_combine_ranked(shape, H: int, plan: Plan, rank_table, topk_w, out):
 
 def pointer_table(ptrs, device) -> torch.Tensor:
     """Device array of raw device addresses (e.g. peers' buffers mapped by
-    ``mep_ipc_open``), for the rank-addressed calls."""
+    ``mep_ipc_open``), for the rank-addressed calls.  The caller keeps the
+    memory behind every address alive while the table is used."""
     return torch.tensor([int(p) for p in ptrs], dtype=torch.int64, device=device)
 
 
