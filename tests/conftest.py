@@ -15,6 +15,20 @@ def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
 
 
+def pytest_sessionstart(session):
+    """On a host with a GPU, make sure the in-tree library is built and up to
+    date with its sources (nvcc, sm_100a; objects that are current are not
+    recompiled).  The tests then load it; nothing falls back to the CPU."""
+    try:
+        import torch
+        have_gpu = torch.cuda.is_available()
+    except Exception:
+        have_gpu = False
+    if have_gpu:
+        from token_dispatch_mep_b200 import build as mep_build
+        mep_build.build()
+
+
 def pytest_collection_modifyitems(config, items):
     try:
         import torch
