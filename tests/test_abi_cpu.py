@@ -199,3 +199,19 @@ def test_rank_pointer_table_keeps_its_buffers_alive():
     del table
     gc.collect()
     assert all(r() is None for r in refs)
+
+
+def test_the_header_is_plain_c_and_the_library_links_from_c(lib, tmp_path):
+    """A C99 program that includes only include/mep.h (no CUDA or C++ header)
+    compiles with -Wall -Werror, links against the library and gets the
+    documented answers from the host-side calls."""
+    import subprocess
+    exe = tmp_path / "abi_from_c"
+    src = os.path.join(ROOT, "tests", "c", "abi_from_c.c")
+    libdir = os.path.dirname(mep.library_path())
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic",
+                    "-I", os.path.join(ROOT, "include"), src, "-o", str(exe),
+                    f"-L{libdir}", "-l:libmep.so", f"-Wl,-rpath,{libdir}"], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert out.returncode == 0, out.stderr
+    assert out.stdout.strip() == "c abi ok"
