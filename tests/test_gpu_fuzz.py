@@ -87,6 +87,16 @@ def test_random_shapes_against_the_oracle(c):
                                       torch.from_numpy(w[r * S:(r + 1) * S].copy()).to(DEV), out_r)
         assert mep.mep_read_status(plan) == 0
         parity.check_plan(plan.host(), pl, f"fuzz hf={home_first}")
+        if not home_first:  # the counts-and-maxvio-only call on the same ids
+            ws = torch.zeros(mep.mep_plan_workspace_bytes(s), dtype=torch.uint8, device=DEV)
+            cnt = torch.empty(E, dtype=torch.int32, device=DEV)
+            mc = torch.empty(1, dtype=torch.int32, device=DEV)
+            mv = torch.empty(1, dtype=torch.float64, device=DEV)
+            stt = torch.full((1,), 7, dtype=torch.int32, device=DEV)
+            mep.mep_maxvio(s, torch.from_numpy(idx).to(DEV), cnt, mc, mv, stt, ws)
+            c_o, m_o, v_o = ora.maxvio(R, S, E, K, idx)
+            assert np.array_equal(cnt.cpu().numpy(), c_o)
+            assert int(mc.item()) == m_o and float(mv.item()) == v_o and int(stt.item()) == 0
         assert np.array_equal(_u16(buf), ora.dispatch(K, pl["src_pair"], _u16(x)))
         ob, ex, ab = ora.combine(pl["slot"], w, _u16(y))
         parity.check_combine(_u16(out), ob, ex, ab, K, "fuzz")

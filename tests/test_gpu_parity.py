@@ -193,7 +193,9 @@ def test_roundrobin_and_adversarial_closed_forms():
 
 
 def test_maxvio_call(ora):
-    for name in ("tiny_r4_e16", "kimi_r64_e896_k16", "skew_r32_zipf1.5"):
+    # tiny: one block; r8: the one-barrier (small tile matrix) form; the
+    # others: two barriers
+    for name in ("tiny_r4_e16", "r8_e64_h2048", "kimi_r64_e896_k16", "skew_r32_zipf1.5"):
         wl = workloads.WORKLOADS[name]
         idx, _ = workloads.routing(wl)
         s = mep.Shape(*wl.shape())
