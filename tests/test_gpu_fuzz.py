@@ -3,7 +3,8 @@ routings -- skewed, duplicate ids inside a token, everything on one expert,
 ids at the edges of [0, E) -- through the C ABI on the GPU, against the
 oracle: both plans bit-exact, dispatch bit-exact, combine and reduce within
 the contract's tolerances, and one rank's token range of the rank-addressed
-calls equal to the whole-range result."""
+calls (dispatch, combine, and the home rank's share of the reduction)
+equal to the whole-range results."""
 import numpy as np
 import pytest
 import torch
@@ -13,6 +14,7 @@ from hypothesis import strategies as st
 import oracle
 import parity
 import token_dispatch_mep_b200 as mep
+from token_dispatch_mep_b200 import ep
 
 pytestmark = pytest.mark.gpu
 
@@ -57,6 +59,7 @@ def case(draw):
 @given(case())
 def test_random_shapes_against_the_oracle(c):
     R, S, E, K, H, P, idx, w, seed = c
+    B = E // R
     ora = oracle.get()
     N, NK, SK = R * S, R * S * K, S * K
     s = mep.Shape(R, S, E, K)
@@ -103,6 +106,21 @@ def test_random_shapes_against_the_oracle(c):
         hexact, habs = ora.reduce(pl["expert_seg_ptr"], G.numpy())
         parity.check_reduce(home.cpu().numpy(), hexact, habs, np.diff(pl["expert_seg_ptr"]), "fuzz")
         assert torch.equal(out_r.view(torch.int16), out[r * S:(r + 1) * S].view(torch.int16))
+        # the home rank r's share of the reduction, from per-rank gradient
+        # buffers (P is often not a multiple of 4: the scalar path)
+        ph = plan.host()
+        rows = ep.max_local_segments(s)
+        grads = []
+        for q in range(R):
+            gq = torch.zeros((rows, P), dtype=torch.float32, device=DEV)
+            for j, (sidx, _, _, _) in enumerate(ep.local_segments(ph, q)):
+                gq[j] = G[sidx].to(DEV)
+            grads.append(gq)
+        home_r = torch.empty((B, P), dtype=torch.float32, device=DEV)
+        gtab = mep.pointer_table([g.data_ptr() for g in grads], DEV)
+        mep.mep_reduce_replica_grads_ranked(s, plan, P, r, gtab, rows, home_r)
+        assert mep.mep_read_status(plan) == 0
+        assert torch.equal(home_r, home[r * B:(r + 1) * B])
         mine = np.unique(pl["slot"][r * S:(r + 1) * S].reshape(-1))
         flat = torch.cat(bufs)
         assert torch.equal(flat[torch.from_numpy(mine).to(DEV).long()].view(torch.int16),
