@@ -37,10 +37,11 @@
 //            offset + rank among equal ids earlier in the warp.  The rank
 //            comes from a peer mask (one ballot per id bit; the lanes holding
 //            the same id) and the popcount of the peers below the lane.
-//            The per-pair work of this loop is what bounds phase 3 on large
-//            workloads (the SM's instruction issue, measured ~0.9 us per
-//            32-pair step of the 32 warps); staging src_pair through shared
-//            memory to coalesce its scattered stores was measured slower.
+//            This loop bounds phase 3 on large workloads: ~0.9 us per 32-pair
+//            step of the 32 warps, nearly the same with its stores removed
+//            (measured in an instrumented copy), so it is bound by the work
+//            per pair, not by memory; staging src_pair through shared memory
+//            to coalesce its scattered stores was measured slower.
 // A warp whose range exceeds its shared-memory id buffer reads its ids again
 // from global memory (L2 hits) in phase 3.
 #include <atomic>
