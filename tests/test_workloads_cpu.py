@@ -61,3 +61,23 @@ def test_reference_arm_prints_one_line(monkeypatch):
     assert line["impl"] == "reference" and line["unit"] == "tokens/s" and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 1
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["metric"] == bench.METRIC
+
+
+def test_roofline_traffic_follows_the_kernel_source(monkeypatch):
+    """bench reports the committed DRAM traffic of a kernel only while its
+    source is the one the counters were taken on, and reads the measured
+    copy peak from MEASURED_PEAKS.json when present."""
+    import os
+
+    import bench
+    rows = [ln.split() for ln in open(os.path.join(bench.ROOT, "profiles", "dram_traffic.txt"))
+            if ln.strip() and not ln.startswith("#")]
+    assert {r[0] for r in rows} >= {"plan", "dispatch", "combine", "reduce"}
+    for name, workload, nbytes, sha, *_ in rows:
+        monkeypatch.setattr(bench, "kernel_sha", lambda n, sha=sha: sha)
+        assert bench.dram_traffic(name, workload) == float(nbytes)        # same source
+        assert bench.dram_traffic(name, "kimi_r64_e896_k16") is None       # no capture there
+        monkeypatch.setattr(bench, "kernel_sha", lambda n: "000000000000")
+        assert bench.dram_traffic(name, workload) is None                  # kernel changed
+    peak, kind = bench.measured_peak()
+    assert peak > 1000 and kind in ("measured", "fallback")
