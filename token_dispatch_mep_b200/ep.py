@@ -149,7 +149,8 @@ class ExchangeGroup:
 
     def barrier(self):
         """This rank's GPU work done, then every rank at the same point."""
-        torch.cuda.current_stream(self.device).synchronize()
+        if self.device.type == "cuda":
+            torch.cuda.current_stream(self.device).synchronize()
         dist.barrier(group=self.group)
 
     def check(self):
