@@ -90,6 +90,9 @@ class Oracle:
         L.ora_prefetch_replicas.restype = None
         L.ora_plan_home_first.argtypes = [ctypes.c_int] * 4 + [_i32p] * 12 + [_i32p, _f64p, _i32p]
         L.ora_plan_home_first.restype = ctypes.c_int
+        L.ora_plan_capped.argtypes = [ctypes.c_int] * 5 + [_i32p] * 12 + [_i32p, _f64p, _i32p,
+                                                                          _i32p, _i32p]
+        L.ora_plan_capped.restype = ctypes.c_int
         self.lib = L
 
     # -- scalars -----------------------------------------------------------
@@ -164,6 +167,40 @@ class Oracle:
         if st:
             raise OracleError(st)
         for n in ("num_seg", "num_replicas", "max_count"):
+            out[n] = int(out[n][0])
+        out["maxvio"] = float(out["maxvio"][0])
+        out["slot"] = out["slot"].reshape(R * S, K)
+        out["rank_seg_idx"] = out["rank_seg_idx"][:out["num_seg"]].copy()
+        return out
+
+    def plan_capped(self, R, S, E, K, B, idx) -> dict:
+        """The capped plan (at most B replica experts per rank when every
+        filler is placed and B >= 3); same fields as ``plan_home_first`` plus
+        ``max_rank_replicas`` (most replica segments on one rank) and
+        ``unplaced`` (fillers left to the stream)."""
+        idx = np.ascontiguousarray(idx, dtype=np.int32).reshape(-1)
+        NK = R * S * K
+        nseg_max = 2 * E + R
+        out = dict(
+            counts=np.zeros(E, np.int32), expert_offset=np.zeros(E + 1, np.int32),
+            slot=np.zeros(NK, np.int32), src_pair=np.zeros(NK, np.int32),
+            seg=np.zeros((nseg_max, 4), np.int32), num_seg=np.zeros(1, np.int32),
+            num_replicas=np.zeros(1, np.int32), rank_seg_ptr=np.zeros(R + 1, np.int32),
+            rank_seg_idx=np.zeros(nseg_max, np.int32),
+            expert_seg_ptr=np.zeros(E + 1, np.int32), replica_seg=np.zeros(nseg_max, np.int32),
+            max_count=np.zeros(1, np.int32), maxvio=np.zeros(1, np.float64),
+            max_rank_replicas=np.zeros(1, np.int32), unplaced=np.zeros(1, np.int32))
+        scratch = np.zeros(12 * E + 10 * R + 1, np.int32)
+        names = ["counts", "expert_offset", "slot", "src_pair", "seg", "num_seg",
+                 "num_replicas", "rank_seg_ptr", "rank_seg_idx", "expert_seg_ptr", "replica_seg",
+                 "max_count"]
+        st = self.lib.ora_plan_capped(R, S, E, K, int(B), _p(idx, _i32p),
+                                      *[_p(out[n], _i32p) for n in names],
+                                      _p(out["maxvio"], _f64p), _p(out["max_rank_replicas"], _i32p),
+                                      _p(out["unplaced"], _i32p), _p(scratch, _i32p))
+        if st:
+            raise OracleError(st)
+        for n in ("num_seg", "num_replicas", "max_count", "max_rank_replicas", "unplaced"):
             out[n] = int(out[n][0])
         out["maxvio"] = float(out["maxvio"][0])
         out["slot"] = out["slot"].reshape(R * S, K)

@@ -521,3 +521,306 @@ int ora_plan_home_first(int R, int S, int E, int K, const int32_t *idx,
     *num_replicas = nr;
     return ORA_OK;
 }
+
+/* ---- capped plan: at most B replica experts per rank ([P1-how] "a small
+ * number of duplicate experts"; [P1-eng] "Key facts": B = E/R for training,
+ * B = 3-4 recommended for inference) ----------------------------------------- *
+ * Reading taken for B: the number of redundant (replica) experts a rank may
+ * host in one step -- the slots of its prefetch buffer for duplicates' weights
+ * -- in addition to its home experts.  (Read instead as the number of distinct
+ * experts a rank may host, the training value E/R would forbid every
+ * duplicate whenever every expert has tokens, and exact S*K balance would be
+ * unreachable: R = 2, E = 2, S*K = 10, T = (15, 5) needs a rank to take pairs
+ * of two experts.)  Every rank still receives exactly S*K slots.
+ *   1. Home fill: each rank takes its home experts in order of increasing
+ *      count (ties: lower id first); expert e keeps h_e = min(T_e, room left)
+ *      pairs home.  F_r = pairs kept on rank r, D_r = S*K - F_r its spare
+ *      room, O_e = T_e - h_e the overflow of e.
+ *   2. Items: experts with O_e > 0 by (O_e descending, e ascending); rooms:
+ *      ranks with D_r > 0 by (D_r descending, r ascending); Dmax = the first
+ *      room's D.
+ *   3. Fillers: the items with O_e < Dmax.  Filler f (f = 0, 1, ... in item
+ *      order) is offered to room f mod Y (Y rooms) in round f / Y; it is
+ *      placed whole, as one replica piece, if the round is below B - 2 and the
+ *      room's space left by earlier rounds holds it.
+ *   4. Stream: the items not placed as fillers, in item order, are cut
+ *      contiguously over the rooms' remaining space, in room order; each
+ *      (item, room) intersection is a replica piece.
+ *   5. Layout: rank r holds its home pieces in ascending expert order (slots
+ *      0 .. F_r - 1), then its replica pieces: fillers by round, then stream
+ *      pieces in stream order.  Expert e's pairs, in (g, k) order: the first
+ *      h_e go home, the others fill its replica pieces in the order the
+ *      pieces were made (its one filler piece, or its stream pieces in room
+ *      order).
+ * When every filler is placed and B >= 3, no rank holds more than B replica
+ * pieces: a room takes at most B - 2 fillers, and the stream items are all at
+ * least Dmax, so a room's remaining space meets at most two of them.
+ * Segments are listed by (expert, rank); rank_seg_idx lists each rank's
+ * segments in slot order.  *max_rank_replicas receives the largest number of
+ * replica segments on one rank, *unplaced the number of fillers not placed.
+ * scratch: 12*E + 10*R + 1 ints. */
+int ora_plan_capped(int R, int S, int E, int K, int B, const int32_t *idx,
+                    int32_t *counts, int32_t *expert_offset, int32_t *slot,
+                    int32_t *src_pair, int32_t *seg, int32_t *num_seg,
+                    int32_t *num_replicas, int32_t *rank_seg_ptr,
+                    int32_t *rank_seg_idx, int32_t *expert_seg_ptr,
+                    int32_t *replica_seg, int32_t *max_count, double *maxvio,
+                    int32_t *max_rank_replicas, int32_t *unplaced,
+                    int32_t *scratch)
+{
+    if (B < 1)
+        return ORA_ERR_ARG;
+    int st = ora_counts(R, S, E, K, idx, counts);
+    if (st)
+        return st;
+    int64_t N = (int64_t)R * S;
+    int64_t C = (int64_t)S * K;
+    int64_t NK = N * K;
+    int Bh = E / R;                               /* home experts per rank */
+    *maxvio = ora_maxvio_from_counts(R, S, E, K, counts, max_count);
+    expert_offset[0] = 0;
+    for (int e = 0; e < E; ++e)
+        expert_offset[e + 1] = expert_offset[e] + counts[e];
+
+    int32_t *h = scratch;                         /* E: pairs kept home */
+    int32_t *O = h + E;                           /* E: overflow */
+    int32_t *item = O + E;                        /* E: items in item order */
+    int32_t *placed_room = item + E;              /* E: room index of a placed filler, else -1 */
+    int32_t *npiece = placed_room + E;            /* E: replica pieces of expert e */
+    int32_t *used = npiece + E;                   /* E: pairs of e placed so far */
+    int32_t *pstart = used + E;                   /* E+1: first piece of e (by expert) */
+    int32_t *F = pstart + E + 1;                  /* R */
+    int32_t *D = F + R;                           /* R */
+    int32_t *room = D + R;                        /* R: rooms in room order */
+    int32_t *left = room + R;                     /* R: space left in room j */
+    int32_t *nrep = left + R;                     /* R: replica pieces on rank r so far */
+    int32_t *rfill = nrep + R;                    /* R: replica slots used on rank r so far */
+    int32_t *hpre = rfill + R;                    /* E: home start of e on its rank */
+    /* pieces, at most E + R of them: expert, rank, size, first slot */
+    int32_t *pe = hpre + E, *pr = pe + E + R, *pn = pr + E + R, *pslot = pn + E + R;
+    (void)pslot;
+
+    /* 1. home fill, smallest home experts first: ord[t] is the home expert of
+     * rank t / Bh's block with (count, id) rank t % Bh */
+    int32_t *ord = O;                             /* borrowed until step 1 ends */
+    for (int r = 0; r < R; ++r) {
+        for (int e = r * Bh; e < (r + 1) * Bh; ++e) {
+            int rank_e = 0;
+            for (int e2 = r * Bh; e2 < (r + 1) * Bh; ++e2)
+                if (counts[e2] < counts[e] || (counts[e2] == counts[e] && e2 < e))
+                    ++rank_e;
+            ord[r * Bh + rank_e] = e;
+        }
+        int64_t fill = 0;
+        for (int t = 0; t < Bh; ++t) {
+            int e = ord[r * Bh + t];
+            int64_t take = counts[e] < C - fill ? counts[e] : C - fill;
+            h[e] = (int32_t)take;
+            fill += take;
+        }
+        F[r] = (int32_t)fill;
+        D[r] = (int32_t)(C - fill);
+    }
+    for (int r = 0; r < R; ++r) {                 /* home pieces in ascending expert order */
+        int64_t at = 0;
+        for (int e = r * Bh; e < (r + 1) * Bh; ++e) {
+            hpre[e] = (int32_t)at;
+            at += h[e];
+        }
+    }
+    for (int e = 0; e < E; ++e)
+        O[e] = counts[e] - h[e];
+
+    /* 2. items and rooms, each by an insertion sort on its key */
+    int X = 0, Y = 0;
+    for (int e = 0; e < E; ++e) {
+        if (O[e] <= 0)
+            continue;
+        int at = X++;
+        while (at > 0 && (O[item[at - 1]] < O[e] ||
+                          (O[item[at - 1]] == O[e] && item[at - 1] > e))) {
+            item[at] = item[at - 1];
+            --at;
+        }
+        item[at] = e;
+    }
+    for (int r = 0; r < R; ++r) {
+        if (D[r] <= 0)
+            continue;
+        int at = Y++;
+        while (at > 0 && (D[room[at - 1]] < D[r] ||
+                          (D[room[at - 1]] == D[r] && room[at - 1] > r))) {
+            room[at] = room[at - 1];
+            --at;
+        }
+        room[at] = r;
+    }
+    for (int j = 0; j < Y; ++j)
+        left[j] = D[room[j]];
+    for (int e = 0; e < E; ++e) {
+        placed_room[e] = -1;
+        npiece[e] = 0;
+    }
+    for (int r = 0; r < R; ++r) {
+        nrep[r] = 0;
+        rfill[r] = F[r];
+    }
+    int np = 0;                                   /* pieces made so far */
+    *unplaced = 0;
+
+    /* 3. fillers, round by round */
+    if (Y > 0) {
+        int32_t dmax = D[room[0]];
+        int f = 0;
+        for (int i = 0; i < X; ++i) {
+            int e = item[i];
+            if (O[e] >= dmax)
+                continue;
+            int j = f % Y, round = f / Y;
+            if (round < B - 2 && left[j] >= O[e]) {
+                placed_room[e] = j;
+                left[j] -= O[e];
+                pstart[e] = np;
+                npiece[e] = 1;
+                pe[np] = e;
+                pr[np] = room[j];
+                pn[np] = O[e];
+                ++np;
+            } else {
+                *unplaced += 1;
+            }
+            ++f;
+        }
+    }
+    /* lay the fillers out: room by room, by round (= the order they were
+     * offered to that room, which is item order) */
+    for (int j = 0; j < Y; ++j) {
+        for (int q = 0; q < np; ++q) {
+            if (pr[q] != room[j])
+                continue;
+            pslot[q] = (int32_t)((int64_t)room[j] * C + rfill[room[j]]);
+            rfill[room[j]] += pn[q];
+            nrep[room[j]] += 1;
+        }
+    }
+    /* 4. the stream: unplaced items against the rooms' remaining space */
+    {
+        int j = 0;
+        int32_t jleft = Y > 0 ? left[0] : 0;
+        for (int i = 0; i < X; ++i) {
+            int e = item[i];
+            if (placed_room[e] >= 0)
+                continue;
+            int32_t need = O[e];
+            while (need > 0) {
+                while (jleft == 0 && j + 1 < Y) { /* next room with space */
+                    ++j;
+                    jleft = left[j];
+                }
+                if (jleft == 0)
+                    return ORA_ERR_DATA;          /* cannot happen: overflow = room */
+                int32_t n = need < jleft ? need : jleft;
+                int r = room[j];
+                if (npiece[e] == 0)
+                    pstart[e] = np;
+                npiece[e] += 1;
+                pe[np] = e;
+                pr[np] = r;
+                pn[np] = n;
+                pslot[np] = (int32_t)((int64_t)r * C + rfill[r]);
+                rfill[r] += n;
+                nrep[r] += 1;
+                ++np;
+                need -= n;
+                jleft -= n;
+            }
+        }
+    }
+    int32_t mx = 0;
+    for (int r = 0; r < R; ++r)
+        if (nrep[r] > mx)
+            mx = nrep[r];
+    *max_rank_replicas = mx;
+
+    /* 5. place every pair, walking pairs in (g, k) order; expert e's replica
+     * pieces are used in the order they were made (piece list order) */
+    for (int e = 0; e < E; ++e)
+        used[e] = 0;
+    for (int64_t pair = 0; pair < NK; ++pair) {
+        int32_t e = idx[pair];
+        int32_t i = used[e]++;
+        int64_t p;
+        if (i < h[e]) {
+            p = (int64_t)(e / Bh) * C + hpre[e] + i;
+        } else {
+            int32_t q = i - h[e];
+            int t = pstart[e];                    /* e's pieces are consecutive */
+            while (q >= pn[t]) {
+                q -= pn[t];
+                ++t;
+            }
+            p = (int64_t)pslot[t] + q;
+        }
+        slot[pair] = (int32_t)p;
+        src_pair[p] = (int32_t)pair;
+    }
+
+    /* 6. segments by (expert, rank): expert e's home piece and replica
+     * pieces, ordered by rank (insertion on the rank) */
+    int32_t ns = 0;
+    for (int e = 0; e < E; ++e) {
+        expert_seg_ptr[e] = ns;
+        int32_t first = ns;
+        for (int t = -1; t < npiece[e]; ++t) {
+            int32_t r, start, n;
+            if (t < 0) {                          /* the home piece */
+                if (h[e] == 0)
+                    continue;
+                r = e / Bh;
+                start = hpre[e];
+                n = h[e];
+            } else {
+                int q2 = pstart[e] + t;
+                r = pr[q2];
+                start = (int32_t)(pslot[q2] - (int64_t)r * C);
+                n = pn[q2];
+            }
+            int32_t q = ns++;
+            while (q > first && seg[4 * (q - 1) + 1] > r) {
+                for (int c = 0; c < 4; ++c)
+                    seg[4 * q + c] = seg[4 * (q - 1) + c];
+                --q;
+            }
+            seg[4 * q + 0] = e;
+            seg[4 * q + 1] = r;
+            seg[4 * q + 2] = start;
+            seg[4 * q + 3] = n;
+        }
+    }
+    expert_seg_ptr[E] = ns;
+    *num_seg = ns;
+    /* each rank's segments in slot order: its segments, by insertion on
+     * their start */
+    int32_t at = 0;
+    for (int r = 0; r < R; ++r) {
+        rank_seg_ptr[r] = at;
+        int32_t first = at;
+        for (int32_t s2 = 0; s2 < ns; ++s2) {
+            if (seg[4 * s2 + 1] != r)
+                continue;
+            int32_t q = at++;
+            while (q > first && seg[4 * rank_seg_idx[q - 1] + 2] > seg[4 * s2 + 2]) {
+                rank_seg_idx[q] = rank_seg_idx[q - 1];
+                --q;
+            }
+            rank_seg_idx[q] = s2;
+        }
+    }
+    rank_seg_ptr[R] = at;
+    int32_t nr = 0;
+    for (int32_t a = 0; a < ns; ++a)
+        if (seg[4 * a + 1] != seg[4 * a] / Bh)
+            replica_seg[nr++] = a;
+    *num_replicas = nr;
+    return ORA_OK;
+}

@@ -619,7 +619,209 @@ def pin_home_first_closed_forms(ora):
     assert a["num_seg"] == 32 and a["num_replicas"] == 31
 
 
+# ---------------------------------------------------- capped schedule
+
+def brute_capped(R, S, E, K, B, idx):
+    """The capped plan as a simulation with pair queues: every expert's pairs
+    queue up in (g, k) order; each rank, taking its home experts smallest
+    count first, keeps the head of each queue while it has room; the
+    overflowing experts line up by overflow (largest first), the ranks with
+    room by room (largest first); the short queues (shorter than the largest
+    room) are offered whole to the rooms in turn, at most B - 2 per room; the
+    queues left over are poured into the rooms' remaining space in line
+    order.  Ranks list home runs by expert, then arrivals in arrival order."""
+    idx = np.asarray(idx).reshape(R * S, K)
+    C, Bh = S * K, E // R
+    queue = [[] for _ in range(E)]
+    for g in range(R * S):
+        for k in range(K):
+            queue[int(idx[g, k])].append(g * K + k)
+    kept = [0] * E
+    for r in range(R):
+        room = C
+        for e in sorted(range(r * Bh, (r + 1) * Bh), key=lambda e: (len(queue[e]), e)):
+            kept[e] = min(len(queue[e]), room)
+            room -= kept[e]
+    home = [[(e, q) for e in range(r * Bh, (r + 1) * Bh) for q in queue[e][:kept[e]]]
+            for r in range(R)]
+    rest = {e: queue[e][kept[e]:] for e in range(E) if len(queue[e]) > kept[e]}
+    line = sorted(rest, key=lambda e: (-len(rest[e]), e))
+    space = {r: C - len(home[r]) for r in range(R) if len(home[r]) < C}
+    rooms = sorted(space, key=lambda r: (-space[r], r))
+    arrivals = {r: [] for r in range(R)}       # (expert, [pairs]) in arrival order
+    poured = []
+    if rooms:
+        dmax = space[rooms[0]]
+        short = [e for e in line if len(rest[e]) < dmax]
+        for f, e in enumerate(short):
+            r = rooms[f % len(rooms)]
+            if f // len(rooms) < B - 2 and space[r] >= len(rest[e]):
+                arrivals[r].append((e, rest[e]))
+                space[r] -= len(rest[e])
+            else:
+                poured.append(e)
+        unplaced = len(poured)
+        poured = [e for e in line if e not in short or e in poured]
+        stream = [(e, q) for e in poured for q in rest[e]]
+        at = 0
+        for r in rooms:
+            take = stream[at:at + space[r]]
+            at += space[r]
+            # group the poured pairs of this room into runs of one expert
+            runs = []
+            for e, q in take:
+                if runs and runs[-1][0] == e:
+                    runs[-1][1].append(q)
+                else:
+                    runs.append((e, [q]))
+            arrivals[r] += runs
+        assert at == len(stream)
+    else:
+        unplaced = 0
+    slot = np.zeros((R * S, K), np.int64)
+    runs = []                                   # [expert, rank, start, count] in slot order
+    for r in range(R):
+        order = [(e, [q]) for e, q in home[r]] + [(e, qs) for e, qs in arrivals[r]]
+        i = 0
+        for e, qs in order:
+            for q in qs:
+                slot[q // K, q % K] = r * C + i
+                if runs and runs[-1][0] == e and runs[-1][1] == r:
+                    runs[-1][3] += 1
+                else:
+                    runs.append([e, r, i, 1])
+                i += 1
+        assert i == C
+    table = sorted(range(len(runs)), key=lambda j: (runs[j][0], runs[j][1]))
+    where = {j: a for a, j in enumerate(table)}
+    seg = [tuple(runs[j]) for j in table]
+    per_rank = [sum(1 for sg in seg if sg[1] == r and sg[1] != sg[0] // Bh) for r in range(R)]
+    return dict(slot=slot, seg=seg, rank_seg_idx=[where[j] for j in range(len(runs))],
+                replica_seg=[a for a, sg in enumerate(seg) if sg[1] != sg[0] // Bh],
+                expert_seg_ptr=[next((a for a, sg in enumerate(seg) if sg[0] >= e), len(seg))
+                                for e in range(E + 1)],
+                rank_seg_ptr=[next((j for j in range(len(runs)) if runs[j][1] >= r), len(runs))
+                              for r in range(R + 1)],
+                max_rank_replicas=max(per_rank), unplaced=unplaced)
+
+
+def check_capped_invariants(pl, R, S, E, K, B, idx):
+    """Exact S*K per rank, each pair once, one expert per run, the static
+    segment bound, replicas never on the home rank, the small-first home
+    fill, and the cap: no rank above B replicas when every filler found a
+    room and B >= 3."""
+    check_home_first_invariants_basic(pl, R, S, E, K, idx)
+    idx = np.asarray(idx).reshape(-1)
+    C, Bh = S * K, E // R
+    counts = np.bincount(idx, minlength=E)
+    ns = pl["num_seg"]
+    seg = np.asarray(pl["seg"])[:ns]
+    kept = np.zeros(E, np.int64)
+    per_rank = np.zeros(R, np.int64)
+    for e, r, st, cnt in seg:
+        if r == e // Bh:
+            kept[e] += cnt
+        else:
+            per_rank[r] += 1
+    assert int(per_rank.max()) == pl["max_rank_replicas"]
+    for r in range(R):                  # smallest home experts are kept whole first
+        order = sorted(range(r * Bh, (r + 1) * Bh), key=lambda e: (counts[e], e))
+        room = C
+        for e in order:
+            assert kept[e] == min(counts[e], room), (r, e)
+            room -= kept[e]
+    if B >= 3 and pl["unplaced"] == 0:
+        assert pl["max_rank_replicas"] <= B
+    overflowing = int((kept < counts).sum())
+    rooms = int(sum(1 for r in range(R) if kept[r * Bh:(r + 1) * Bh].sum() < C))
+    assert pl["num_replicas"] <= max(0, overflowing + rooms - 1)
+
+
+def check_home_first_invariants_basic(pl, R, S, E, K, idx):
+    idx = np.asarray(idx).reshape(-1)
+    NK, C, Bh = R * S * K, S * K, E // R
+    slot = np.asarray(pl["slot"]).reshape(-1).astype(np.int64)
+    src = np.asarray(pl["src_pair"]).astype(np.int64)
+    assert np.array_equal(np.sort(slot), np.arange(NK))
+    assert np.array_equal(src[slot], np.arange(NK))
+    ns = pl["num_seg"]
+    seg = np.asarray(pl["seg"])[:ns]
+    assert ns <= E + R - 1
+    assert np.array_equal(np.bincount(seg[:, 1], weights=seg[:, 3], minlength=R), np.full(R, C))
+    e_of_p = idx[src]
+    for e, r, st, cnt in seg:
+        assert np.all(e_of_p[r * C + st: r * C + st + cnt] == e)
+    assert len({(int(e), int(r)) for e, r, _, _ in seg}) == ns      # one run per (expert, rank)
+
+
+def _check_capped_equal(pl, ref, what=""):
+    _check_hf_equal(pl, ref, what)
+    assert pl["max_rank_replicas"] == ref["max_rank_replicas"], what
+    assert pl["unplaced"] == ref["unplaced"], what
+
+
+def pin_capped(ora):
+    gd = load_golden("example_d_capped.json")
+    idx = np.array(gd["idx"], np.int32)
+    for c in gd["cases"]:
+        pl = ora.plan_capped(gd["R"], gd["S"], gd["E"], gd["K"], c["B"], idx)
+        assert list(pl["counts"]) == gd["counts"]
+        assert pl["maxvio"] == gd["maxvio_num"] / gd["maxvio_den"] - 1.0
+        assert pl["slot"].tolist() == c["slot"], c["B"]
+        assert pl["seg"][:pl["num_seg"]].tolist() == c["segments"], c["B"]
+        assert list(pl["replica_seg"][:pl["num_replicas"]]) == c["replica_seg"]
+        assert list(pl["rank_seg_ptr"]) == c["rank_seg_ptr"]
+        assert list(pl["rank_seg_idx"]) == c["rank_seg_idx"]
+        assert list(pl["expert_seg_ptr"]) == c["expert_seg_ptr"]
+        assert pl["max_rank_replicas"] == c["max_rank_replicas"]
+        assert pl["unplaced"] == c["unplaced"]
+    rng = np.random.default_rng(43)
+    for (R, S, E, K) in SMALL_SHAPES:
+        for distinct, skew in ((True, 0.0), (True, 2.5), (False, 0.0), (False, 4.0)):
+            idx = _random_idx(rng, R, S, E, K, distinct, skew)
+            for B in (1, 2, 3, 4, E // R):
+                pl = ora.plan_capped(R, S, E, K, B, idx)
+                _check_capped_equal(pl, brute_capped(R, S, E, K, B, idx), str((R, S, E, K, B)))
+                check_capped_invariants(pl, R, S, E, K, B, idx)
+    import workloads
+    for name, S in (("kimi_r64_e896_k16", 23), ("skew_r32_zipf1.5", 61), ("r8_e64_h2048", 97),
+                    ("skew_r32_uniform", 40)):
+        wl = workloads.reduced(workloads.WORKLOADS[name], S=S)
+        idx, _ = workloads.routing(wl)
+        for B in (3, 4, wl.E // wl.R):
+            pl = ora.plan_capped(wl.R, wl.S, wl.E, wl.K, B, idx)
+            check_capped_invariants(pl, wl.R, wl.S, wl.E, wl.K, B, idx)
+            _check_capped_equal(pl, brute_capped(wl.R, wl.S, wl.E, wl.K, B, idx), name)
+
+
+def pin_capped_closed_forms(ora):
+    """Round-robin routing fills every rank from home: no replica at all.
+    Adversarial routing (every token on experts 0..7, R = 32, E = 256, S*K =
+    32768): rank 0 keeps 32768 pairs of expert 0 (ties go to the lower id),
+    experts 1..7 overflow whole (131072 each) and expert 0 by 98304; the 31
+    empty ranks are rooms of 32768; no overflow is below the largest room, so
+    the stream gives experts 1..7 four ranks each (1-4, ..., 25-28) and expert
+    0 ranks 29-31: 31 replicas, one per rank."""
+    import workloads
+    for (R, S, E, K) in [(4, 64, 16, 2), (8, 512, 64, 6), (2, 3, 6, 4)]:
+        idx, _ = workloads.roundrobin_routing(R, S, E, K)
+        for B in (1, 4):
+            pl = ora.plan_capped(R, S, E, K, B, idx)
+            assert pl["num_replicas"] == 0 and pl["max_rank_replicas"] == 0
+            assert np.array_equal(pl["slot"], ora.plan(R, S, E, K, idx)["slot"])
+    R, S, E, K = 32, 4096, 256, 8
+    idx = np.argsort(-np.random.default_rng(0).standard_normal((R * S, K)), axis=1).astype(np.int32)
+    pl = ora.plan_capped(R, S, E, K, 4, idx)
+    assert pl["num_seg"] == 32 and pl["num_replicas"] == 31 and pl["max_rank_replicas"] == 1
+    want = [(0, 0, 0, 32768)] + [(0, r, 0, 32768) for r in (29, 30, 31)]
+    for e in range(1, 8):
+        want += [(e, 4 * (e - 1) + 1 + j, 0, 32768) for j in range(4)]
+    want.sort()
+    assert [tuple(x) for x in pl["seg"][:32].tolist()] == want
+
+
 ALL_PINS = [pin_bf16_widen, pin_bf16_rounding, pin_plan_golden, pin_plan_bruteforce,
             pin_plan_invariants, pin_closed_forms, pin_errors, pin_dispatch,
             pin_combine, pin_reduce, pin_combine_backward, pin_dispatch_backward,
-            pin_prefetch_replicas, pin_home_first, pin_home_first_closed_forms]
+            pin_prefetch_replicas, pin_home_first, pin_home_first_closed_forms,
+            pin_capped, pin_capped_closed_forms]

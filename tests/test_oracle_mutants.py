@@ -73,6 +73,25 @@ MUTANTS = {
         "p = (int64_t)r * C + F[r] + (q - D[r]);", "p = (int64_t)r * C + (q - D[r]);"),
     "home_first_replica_flag_by_slot_rank": (
         "if (seg[4 * a + 1] != seg[4 * a] / B)", "if (seg[4 * a + 1] != seg[4 * a] % R)"),
+    "capped_home_fill_largest_first": (
+        "if (counts[e2] < counts[e] || (counts[e2] == counts[e] && e2 < e))",
+        "if (counts[e2] > counts[e] || (counts[e2] == counts[e] && e2 < e))"),
+    "capped_items_ascending": (
+        "while (at > 0 && (O[item[at - 1]] < O[e] ||",
+        "while (at > 0 && (O[item[at - 1]] > O[e] ||"),
+    "capped_rooms_ascending": (
+        "while (at > 0 && (D[room[at - 1]] < D[r] ||",
+        "while (at > 0 && (D[room[at - 1]] > D[r] ||"),
+    "capped_one_round_too_many": (
+        "if (round < B - 2 && left[j] >= O[e]) {", "if (round < B - 1 && left[j] >= O[e]) {"),
+    "capped_filler_threshold_inclusive": (
+        "if (O[e] >= dmax)\n                continue;", "if (O[e] > dmax)\n                continue;"),
+    "capped_replicas_over_home_slots": ("rfill[r] = F[r];", "rfill[r] = 0;"),
+    "capped_last_pairs_stay_home": (
+        "        if (i < h[e]) {\n            p = (int64_t)(e / Bh) * C + hpre[e] + i;\n"
+        "        } else {\n            int32_t q = i - h[e];",
+        "        if (i >= O[e]) {\n            p = (int64_t)(e / Bh) * C + hpre[e] + (i - O[e]);\n"
+        "        } else {\n            int32_t q = i;"),
 }
 
 
