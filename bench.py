@@ -110,7 +110,7 @@ def dram_traffic(name: str, workload: str):
 
 class ClockSampler:
     """Samples the SM clock and the clock-event reasons with NVML every
-    ~20 ms in a background thread (reads only; changes no setting)."""
+    ~10 ms in a background thread (reads only; changes no setting)."""
 
     BITS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
             0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
@@ -150,7 +150,7 @@ class ClockSampler:
                         self.reasons.add(name)
             except Exception:
                 pass
-            time.sleep(0.02)
+            time.sleep(0.01)
 
     def start(self):
         if self._h is not None:
@@ -180,33 +180,68 @@ def max_over_ranks(value: float, world: int, device) -> float:
     return float(t.item())
 
 
+def rank_replicas_max(plan_host: dict, experts_per_rank: int, R: int) -> int:
+    """Most replica segments on one rank, from a host copy of a plan."""
+    seg = np.asarray(plan_host["seg"])[:plan_host["num_seg"]]
+    rep = seg[seg[:, 1] != seg[:, 0] // experts_per_rank]
+    return int(np.bincount(rep[:, 1], minlength=R).max()) if len(rep) else 0
+
+
 def whole_job_rate(tokens_per_rank: int, world: int, ms: float) -> float:
     """Tokens per second of all replicas together, timed by the slowest."""
     return tokens_per_rank * world / (ms * 1e-3)
 
 
+# ------------------------------------------------------------ config
+
+L2_NOTE = ("flushed between steps, outside the events: a 512 MB write, then a 512 MB read "
+           "that writes the fill's dirty lines back")
+
+
+def bench_config(wl, world: int) -> dict:
+    """The workload's `config`, identical in both arms' lines."""
+    return {"workload": wl.name, "R": wl.R, "S": wl.S, "E": wl.E, "K": wl.K, "H": wl.H,
+            "P": wl.P,
+            "step": "plan+dispatch+combine" + ("+replica-grad reduce" if wl.P else ""),
+            "l2": L2_NOTE, "parallelism": f"replicas x{world}"}
+
+
 # ------------------------------------------------------------ CPU oracle leg
+
+# Host bytes above which the combine sample reads a folded copy of the
+# expert outputs (see oracle_throughput).
+Y_HOST_LIMIT = 2 << 30
+
 
 def oracle_throughput(wl, target_seconds: float, host=None):
     """Time the oracle, as it stands, on a bounded sample of the workload:
-    the whole plan, dispatch and combine of the first n tokens, the reduction
-    of the first c gradient columns; scaled to tokens per second of the full
-    step.  Single-threaded C."""
+    the whole plan; dispatch of the first n slots and combine of the first n
+    tokens, both through the plan's own src_pair / slot (so rows are read
+    and written in the plan's scattered order); the reduction of the first c
+    gradient columns; scaled to tokens per second of the full step.
+    Single-threaded C.  Where the expert outputs would exceed Y_HOST_LIMIT
+    bytes of host memory, the combine reads them from M rows (M*H*2 bytes
+    just under the limit, far larger than the host's caches) at slot mod M."""
     import oracle
+    import torch
     ora = oracle.get()
-    R, S, E, K, H, P, N = wl.R, wl.S, wl.E, wl.K, wl.H, wl.P, wl.N
+    R, S, E, K, H, P, N, NK = wl.R, wl.S, wl.E, wl.K, wl.H, wl.P, wl.N, wl.NK
     if host is None:
         idx, w = workloads.routing(wl)
         host = dict(idx=idx, w=w)
     idx, w = host["idx"], host["w"]
+    pl = ora.plan(R, S, E, K, idx)
     # size the samples from the budget (about 12 ns per combine term, 3 ns per
     # reduced element on this kind of host core)
     per_tok = K * H * 12.5e-9
     n_tok = int(max(1, min(N, (0.5 * target_seconds) / per_tok)))
-    x = workloads.hidden(n_tok, H, seed=1).view(__import__("torch").int16).numpy().view(np.uint16)
-    y = workloads.expert_outputs(n_tok * K, H, seed=2).view(__import__("torch").int16).numpy().view(np.uint16)
-    pairs = np.arange(n_tok * K, dtype=np.int32)
-    local_slot = np.arange(n_tok * K, dtype=np.int32).reshape(n_tok, K)
+    n_slot = min(NK, n_tok * K)
+    u16 = lambda t: t.view(torch.int16).numpy().view(np.uint16)
+    x = u16(workloads.hidden(N, H, seed=1))
+    m_rows = int(min(NK, max(1, Y_HOST_LIMIT // (2 * H))))
+    y = u16(workloads.expert_outputs(m_rows, H, seed=2))
+    src = np.ascontiguousarray(pl["src_pair"][:n_slot])
+    slot = np.ascontiguousarray(pl["slot"][:n_tok] % m_rows).astype(np.int32)
     n_col = int(max(1, min(P, (0.4 * target_seconds) / (3.2e-9 * (wl.seg_rows + E))))) if P else 0
     G = workloads.seg_grads(wl.seg_rows, n_col, seed=3).numpy() if P else None
     # Where the sample is the whole workload and takes less than the budget,
@@ -217,24 +252,27 @@ def oracle_throughput(wl, target_seconds: float, host=None):
         pl = ora.plan(R, S, E, K, idx)
         t_plan = time.perf_counter() - t0
         t0 = time.perf_counter()
-        ora.dispatch(K, pairs, x)
+        ora.dispatch(K, src, x)
         t_disp = time.perf_counter() - t0
         t0 = time.perf_counter()
-        ora.combine(local_slot, w[:n_tok], y)
+        ora.combine(slot, w[:n_tok], y)
         t_comb = time.perf_counter() - t0
         t_red = 0.0
         if P:
             t0 = time.perf_counter()
             ora.reduce(pl["expert_seg_ptr"], G)
             t_red = time.perf_counter() - t0
-        t_step = t_plan + (t_disp + t_comb) * (N / n_tok) + (t_red * (P / n_col) if P else 0.0)
+        t_step = (t_plan + t_disp * (NK / n_slot) + t_comb * (N / n_tok)
+                  + (t_red * (P / n_col) if P else 0.0))
         reps.append((t_step, dict(plan=t_plan, dispatch=t_disp, combine=t_comb, reduce=t_red)))
         measured += t_plan + t_disp + t_comb + t_red
     reps.sort(key=lambda r: r[0])
     t_step, parts = reps[len(reps) // 2]
-    sample = (f"whole plan; dispatch+combine of {n_tok}/{N} tokens; "
-              f"reduce of {n_col}/{P} gradient columns; scaled to the full step; "
-              f"median of {len(reps)} repetition(s)")
+    fold = "" if m_rows == NK else f" (expert outputs folded to {m_rows} rows: slot mod {m_rows})"
+    sample = (f"whole plan; dispatch of {n_slot}/{NK} slots via the plan's src_pair; "
+              f"combine of {n_tok}/{N} tokens via the plan's slots{fold}; "
+              + (f"reduce of {n_col}/{P} gradient columns; " if P else "")
+              + f"scaled to the full step; median of {len(reps)} repetition(s)")
     return dict(value=N / t_step, t_step=t_step, sample=sample, measured_s=measured,
                 repetitions=len(reps), parts=parts)
 
@@ -257,8 +295,8 @@ def run_reference(args):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": t * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": wl.name, "R": wl.R, "S": wl.S, "E": wl.E, "K": wl.K,
-                   "H": wl.H, "P": wl.P},
+        "config": bench_config(wl, args.gpus),
+        "timing": "host wall clock (time.perf_counter) around each oracle call",
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                          "sample": vals[0]["sample"]},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -351,7 +389,6 @@ def main():
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    clocks = sampler.stop()
     st = mep.mep_read_status(plan)
     if st != 0:
         raise RuntimeError(f"device status {mep.mep_status_string(st)}")
@@ -385,6 +422,7 @@ def main():
 
     # ---- the home-first (low-replica) plan: latency and replica count
     home_first = None
+    capped = None
     if not args.no_backward:
         hf = mep.Plan(s, dev)
         hts = []
@@ -403,6 +441,29 @@ def main():
         home_first = {"plan_us": float(np.median([a.elapsed_time(b) for a, b in hts])) * 1e3,
                       "num_replicas": hh["num_replicas"], "num_seg": hh["num_seg"],
                       "num_replicas_contiguous": plan.host()["num_replicas"]}
+        # the capped plan at the pages' two values of B (training E/R,
+        # inference 4): latency, replicas, and the most replicas on one rank
+        capped = {}
+        for B in (E // R, 4):
+            mr = torch.zeros(1, dtype=torch.int32, device=dev)
+            cts = []
+            for it in range(3 + 20):
+                flush_l2()
+                h0, h1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                h0.record()
+                mep.mep_plan_capped(s, B, idx, hf, mr)
+                h1.record()
+                if it >= 3:
+                    cts.append((h0, h1))
+            torch.cuda.synchronize()
+            if mep.mep_read_status(hf) != 0:
+                raise RuntimeError("device status not OK after the capped plan")
+            hc = hf.host()
+            capped[f"B={B}"] = {"plan_us": float(np.median([a.elapsed_time(b) for a, b in cts])) * 1e3,
+                                "num_replicas": hc["num_replicas"], "num_seg": hc["num_seg"],
+                                "max_rank_replicas": int(mr.item())}
+        home_first["max_rank_replicas"] = rank_replicas_max(hh, E // R, R)
+        home_first["max_rank_replicas_contiguous"] = rank_replicas_max(plan.host(), E // R, R)
         del hf
 
     # ---- the same step captured once in a CUDA graph and replayed
@@ -432,6 +493,8 @@ def main():
             raise RuntimeError("device status not OK after graph replays")
         graph = {"ms_per_step": gms, "value": whole_job_rate(N, world, gms), "unit": "tokens/s"}
         del cg
+    # the clock record spans both timed loops (eager and graph replay)
+    clocks = sampler.stop()
 
     # ---- backward of combine and dispatch and the replica weight prefetch
     # (each timed alone, not part of the step)
@@ -567,13 +630,9 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": wl.name, "R": R, "S": S, "E": E, "K": K, "H": H, "P": P,
-                       "step": "plan+dispatch+combine+replica-grad reduce",
-                       "l2": ("flushed between steps, outside the events: a 512 MB write, then a "
-                              "512 MB read that writes the fill's dirty lines back"),
-                       "timing": ("CUDA-graph replay of the captured step, events around each replay"
-                                  if graph is not None else "eager launches, events around each kernel"),
-                       "parallelism": f"replicas x{world}"},
+            "config": bench_config(wl, world),
+            "timing": ("CUDA-graph replay of the captured step, events around each replay"
+                       if graph is not None else "eager launches, events around each kernel"),
             "roofline": roofline,
             "cpu_baseline": cpu,
             "e2e": e2e,
@@ -583,6 +642,7 @@ def main():
             "backward_kernels": backward,
             "graph_replay": graph,
             "home_first_plan": home_first,
+            "capped_plan": capped,
             "eager": eager,
             "kernels": kernels,
             "plan_us": stage_ms["plan"] * 1e3,

@@ -65,7 +65,7 @@ extern "C" {
 #define MEP_API
 #endif
 
-#define MEP_VERSION 3
+#define MEP_VERSION 4
 #define MEP_MAX_EXPERTS 1024      /* E <= 1024 */
 #define MEP_MAX_RANKS 1024        /* R <= 1024 */
 #define MEP_MAX_HIDDEN 32768      /* H <= 32768 bf16 elements per row */
@@ -170,6 +170,85 @@ MEP_API mep_status_t mep_plan(mep_shape_t shape, const int32_t *topk_idx,
 MEP_API mep_status_t mep_plan_home_first(mep_shape_t shape, const int32_t *topk_idx,
                                          const mep_plan_t *plan, void *ws, size_t ws_bytes,
                                          void *stream);
+
+/* The capped plan: at most B replica experts per rank ("How MoonEP works": a
+ * small number of duplicate experts; "Key facts about the release": B = E/R
+ * for training, 3-4 recommended for inference).  The pages do not define B;
+ * this library reads it as the number of replica (duplicate) experts a rank
+ * may host besides its home experts -- the slots of its buffer for
+ * duplicates' weights.  Same outputs as mep_plan (and the same workspace);
+ * the pages fix no algorithm, this is the one this library takes:
+ *   1. rank r keeps its home experts' pairs, smallest expert (by T_e, ties to
+ *      the lower id) first: expert e keeps h_e = min(T_e, room left);
+ *   2. items = experts that overflow, by overflow descending (ties: lower
+ *      id); rooms = ranks with spare room, by room descending (ties: lower
+ *      rank); Dmax = the largest room;
+ *   3. items with overflow below Dmax are fillers: filler f (in item order)
+ *      is offered to room f mod Y (Y rooms) in round f / Y and placed whole,
+ *      as one replica piece, if the round is below B - 2 and the room's space
+ *      left holds it;
+ *   4. the other items, in item order, are cut contiguously over the rooms'
+ *      space left, in room order;
+ *   5. rank r's slots hold its home pieces (ascending expert), then its
+ *      fillers (by round), then its stream pieces (stream order); expert e's
+ *      pairs in (g, k) order fill its home piece (the first h_e), then its
+ *      replica pieces in the order they were made.
+ * Every rank receives exactly S*K slots.  When every filler is placed and
+ * B >= 3, no rank hosts more than B replicas (a room takes at most B - 2
+ * fillers, and the stream items are all at least Dmax, so a room's space
+ * left meets at most two of them); otherwise the cap may be exceeded.
+ *   B                  >= 1 (values above E + 2 act as E + 2).
+ *   max_rank_replicas  int32 [1] device out: the most replica segments on
+ *                      one rank; compare it with B.
+ * Segments are listed by (expert, rank); rank_seg_idx lists each rank's
+ * segments in slot order; expert_offset is the exclusive prefix sum of
+ * counts.  At most E + R - 1 segments. */
+MEP_API mep_status_t mep_plan_capped(mep_shape_t shape, int32_t B, const int32_t *topk_idx,
+                                     const mep_plan_t *plan, int32_t *max_rank_replicas,
+                                     void *ws, size_t ws_bytes, void *stream);
+
+/* The schedules a plan can follow (mep_plan_rank). */
+typedef enum {
+    MEP_SCHEDULE_CONTIGUOUS = 0,  /* mep_plan */
+    MEP_SCHEDULE_HOME_FIRST = 1,  /* mep_plan_home_first */
+    MEP_SCHEDULE_CAPPED = 2       /* mep_plan_capped */
+} mep_schedule_t;
+
+/* One rank's histogram, the input of the plan's one exchange between ranks
+ * ("The problem MoonEP targets": T_e counts the tokens routed to expert e).
+ *   local_idx  int32 [S, K], the rank's own top-K expert ids.
+ *   counts     int32 [E] out: how many of those S*K pairs go to each expert.
+ *   status     int32 [1] out: device error word, cleared by this call
+ *              (MEP_ERR_DEVICE_DATA for an id outside [0, E)).
+ *   ws         workspace of mep_plan_workspace_bytes(shape) bytes.
+ * On a multi-GPU system every rank all-gathers these E-vectors (R x E int32:
+ * 229 KB on the R = 64, E = 896 shape) and calls mep_plan_rank. */
+MEP_API mep_status_t mep_rank_histogram(mep_shape_t shape, const int32_t *local_idx,
+                                        int32_t *counts, int32_t *status, void *ws,
+                                        size_t ws_bytes, void *stream);
+
+/* One rank's share of the plan, from the gathered histograms ("How MoonEP
+ * works": every rank computes the same schedule from the current routing).
+ *   schedule       a mep_schedule_t; B and max_rank_replicas as in
+ *                  mep_plan_capped (ignored, may be 0 / NULL, otherwise).
+ *   rank           0 <= rank < R: the rank whose tokens local_idx holds
+ *                  (global tokens rank*S .. rank*S + S - 1).
+ *   local_idx      int32 [S, K].
+ *   rank_counts    int32 [R, E] device: row r = mep_rank_histogram of rank
+ *                  r's ids.  Row `rank` must equal this rank's own histogram
+ *                  (checked on the device: MEP_ERR_DEVICE_DATA otherwise).
+ *   plan           written exactly as the whole-range call of the same
+ *                  schedule writes it, except slot and src_pair: slot rows
+ *                  rank*S .. rank*S + S - 1 (this rank's pairs) and src_pair
+ *                  at those pairs' slots; other entries are not touched.
+ * A pair's place among its expert's pairs is the number of pairs of that
+ * expert on lower ranks (a prefix of the gathered columns; tokens are
+ * numbered rank-major) plus its place among the rank's own, so every rank's
+ * tables equal the whole-range plan's bit for bit. */
+MEP_API mep_status_t mep_plan_rank(mep_shape_t shape, int32_t schedule, int32_t B, int32_t rank,
+                                   const int32_t *local_idx, const int32_t *rank_counts,
+                                   const mep_plan_t *plan, int32_t *max_rank_replicas,
+                                   void *ws, size_t ws_bytes, void *stream);
 
 /* Zero-copy dispatch into the static receive buffer ("Why this matters to
  * engineers": each row is copied directly to its final expert-ordered slot).
@@ -352,16 +431,45 @@ MEP_API mep_status_t mep_dispatch_backward(mep_shape_t shape, int32_t H, const m
  * loads the library until the process exits.  It holds the workspace of
  * the largest shape the library accepts (E = MEP_MAX_EXPERTS); a shape beyond
  * the shape rules is rejected with MEP_ERR_INVALID_ARG, and a workspace that
- * would not fit the array with MEP_ERR_WORKSPACE, before anything runs.  The first
- * call on a device looks up that array's device address (make that call
- * before any stream capture on the device).  Each call clears the array's
- * barrier words with a 256-byte memset on `stream`, then launches the plan.
+ * would not fit the array with MEP_ERR_WORKSPACE, before anything runs; every
+ * argument check of mep_plan also runs before anything is queued.  The first
+ * call in a CUDA context of a device looks up that array's device address in
+ * that context (make that call before any stream capture on the device); a
+ * call in a new context of the device, e.g. after cudaDeviceReset, looks it up
+ * again.  Each call clears the array's barrier words with a 256-byte memset on
+ * `stream`, then launches the plan.
  * The array is shared by all calls on a device: calls that overlap on the GPU
  * (e.g. on two streams with no ordering between them) race and give
  * undefined plans.  Allocates nothing and frees nothing. */
 #define MEP_NOALLOC_SCRATCH_BYTES (256u + 1024u * 1024u * 4u)
 MEP_API mep_status_t mep_plan_noalloc(mep_shape_t shape, const int32_t *topk_idx,
                                       const mep_plan_t *plan, void *stream);
+
+/* A barrier between the ranks of an expert-parallel group, on the device, in
+ * place of a host round trip between the exchange's phases ("Why this
+ * matters to engineers": no per-layer host synchronisation).
+ *   peer_flags  device array of R device pointers (8-byte aligned); pointer p
+ *               addresses rank p's R flag words (uint32, 4-byte aligned), in
+ *               rank p's memory and mapped into this process (mep_ipc_open),
+ *               or any device-visible memory.
+ *   my_flags    this rank's own R flag words (the array peer_flags[rank]
+ *               addresses, as this process sees it).
+ *   rank        0 <= rank < R <= MEP_MAX_RANKS.
+ *   epoch       this crossing's number; use 1, 2, 3, ... on every rank (the
+ *               words start at 0; comparisons are modulo 2^32).
+ *   status      int32 [1] device word: MEP_ERR_TIMEOUT if some rank's word did
+ *               not reach `epoch` within mep_get_wait_limit_ns, and
+ *               MEP_ERR_DEVICE_DATA for a NULL or misaligned peer pointer
+ *               (first error wins; the word is not cleared).
+ * One kernel: after every earlier write of `stream` is made visible system-
+ * wide, it stores `epoch` into word `rank` of every rank's array (release,
+ * system scope), then waits until all R words of my_flags have reached
+ * `epoch` (acquire, system scope).  Later work on `stream` then sees every
+ * rank's writes from before its own arrival.  Every rank must call it with
+ * the same epochs, in the same order. */
+MEP_API mep_status_t mep_rank_barrier(uint32_t *const *peer_flags, uint32_t *my_flags, int32_t R,
+                                      int32_t rank, uint32_t epoch, int32_t *status,
+                                      void *stream);
 
 /* Synchronises `stream` and returns the plan's device status word (MEP_OK if
  * every call so far on this plan ran clean), or MEP_ERR_CUDA if the copy
@@ -372,7 +480,8 @@ MEP_API mep_status_t mep_read_status(const mep_plan_t *plan, void *stream);
 MEP_API const char *mep_status_string(mep_status_t status);
 
 /* Upper bound, in nanoseconds of the GPU global timer, on every device-side
- * wait (the grid barriers of mep_plan and mep_maxvio).  A wait that runs out
+ * wait (the grid barriers of the plan calls and the waits of
+ * mep_rank_barrier).  A wait that runs out
  * records MEP_ERR_TIMEOUT and the kernel returns.  Process-wide; default 1e9
  * (one second); values below 1000 are raised to 1000. */
 MEP_API void mep_set_wait_limit_ns(uint64_t ns);

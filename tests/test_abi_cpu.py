@@ -43,7 +43,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_version_and_strings(lib):
-    assert mep.mep_version() == 3
+    assert mep.mep_version() == 4
     for code, name in mep.STATUS.items():
         assert mep.mep_status_string(code)
     assert mep.mep_status_string(99) == "unknown status"
@@ -115,6 +115,14 @@ def test_host_side_rejections_launch_nothing(lib):
     i4 = vp(0x100000)
     assert L.mep_maxvio(s, i4, i4, i4, vp(0x100004), i4, good, 1 << 30, None) == 2
     assert L.mep_maxvio(s, i4, i4, i4, good, i4, good, 8, None) == 3
+    # the capped plan: B >= 1, a cap output, then the plan rules
+    assert L.mep_plan_capped(s, 0, good, ctypes.byref(p), i4, good, 1 << 30, None) == 1
+    assert L.mep_plan_capped(s, 4, good, ctypes.byref(p), None, good, 1 << 30, None) == 1
+    assert L.mep_plan_capped(s, 4, good, ctypes.byref(p), vp(0x100002), good, 1 << 30, None) == 2
+    assert L.mep_plan_capped(s, 4, good, ctypes.byref(q), i4, good, 1 << 30, None) == 2
+    assert L.mep_plan_capped(s, 4, good, ctypes.byref(p), i4, good, 16, None) == 3
+    assert L.mep_plan_capped(mep.Shape(2, 4, 3, 2), 4, good, ctypes.byref(p), i4, good,
+                             1 << 30, None) == 1
 
 
 def test_package_has_no_cpu_fallback(tmp_path, monkeypatch):

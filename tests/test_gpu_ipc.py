@@ -60,7 +60,8 @@ def _rank_main(rank, world, port, schedule, q):
         G = workloads.seg_grads(wl.seg_rows, P, seed=3)
         mine = slice(rank * S, (rank + 1) * S)
 
-        grp = ep.ExchangeGroup(mep.Shape(R, S, E, K), H, P, device=dev, schedule=schedule)
+        grp = ep.ExchangeGroup(mep.Shape(R, S, E, K), H, P, device=dev, schedule=schedule,
+                               B=4 if schedule == "capped" else 0)
         plan = grp.make_plan(torch.from_numpy(idx[mine].copy()))
         recv = grp.dispatch(x[mine].to(dev))
         grp.y.copy_(y[rank * SK:(rank + 1) * SK].to(dev))        # this rank's expert outputs
@@ -73,9 +74,18 @@ def _rank_main(rank, world, port, schedule, q):
         grp.check()
 
         ora = oracle.get()
-        pl = (ora.plan if schedule == "contiguous" else ora.plan_home_first)(R, S, E, K, idx)
+        if schedule == "contiguous":
+            pl = ora.plan(R, S, E, K, idx)
+        elif schedule == "home_first":
+            pl = ora.plan_home_first(R, S, E, K, idx)
+        else:
+            pl = ora.plan_capped(R, S, E, K, 4, idx)
         res = {}
-        res["plan"] = bool(np.array_equal(ph["slot"].reshape(-1), pl["slot"].reshape(-1)))
+        # this rank's own pairs' slots and every table (the plan came from the
+        # gathered histograms: the other ranks' slot rows are not this rank's)
+        res["plan"] = bool(np.array_equal(ph["slot"][mine], pl["slot"][mine]) and
+                           grp.gathered_bytes == R * E * 4)
+        parity.check_plan(dict(ph, slot=pl["slot"], src_pair=pl["src_pair"]), pl, f"rank {rank}")
         want = ora.dispatch(K, pl["src_pair"], u16(x))[rank * SK:(rank + 1) * SK]
         res["dispatch"] = bool(np.array_equal(u16(recv), want))
         ob, ex, ab = ora.combine(pl["slot"], w, u16(y))
@@ -102,7 +112,7 @@ def _rank_main(rank, world, port, schedule, q):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("schedule", ["contiguous", "home_first"])
+@pytest.mark.parametrize("schedule", ["contiguous", "home_first", "capped"])
 def test_two_process_exchange_over_ipc(schedule):
     world = 2
     ctx = mp.get_context("spawn")

@@ -61,6 +61,11 @@ def test_reference_arm_prints_one_line(monkeypatch):
     assert line["impl"] == "reference" and line["unit"] == "tokens/s" and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 1
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["metric"] == bench.METRIC
+    # the same config keys and values as the GPU arm's line
+    assert line["config"] == bench.bench_config(workloads.WORKLOADS["tiny_r4_e16"], 1)
+    # the oracle runs through the plan's own slots, not sequential ones
+    assert "via the plan's src_pair" in line["cpu_baseline"]["sample"]
+    assert "via the plan's slots" in line["cpu_baseline"]["sample"]
 
 
 def test_roofline_traffic_follows_the_kernel_source(monkeypatch):

@@ -32,6 +32,26 @@ def test_rejects_shapes_beyond_the_limits():
     assert L.mep_plan_noalloc(mep.Shape(2, 4, 8, 2), idx, None, None) == 1
 
 
+def test_checks_every_plan_field_before_queueing_anything():
+    """A NULL or misaligned plan field is reported by the host-side checks,
+    before the scratch memset is queued: these calls reach no CUDA API at all
+    (they run here without a GPU)."""
+    L = mep.load_library()
+    fields = [f for f, _ in mep._PlanStruct._fields_]
+    aligned = {f: 0x100000 + 0x1000 * i for i, f in enumerate(fields)}
+    s = mep.Shape(2, 4, 8, 2)
+    idx = ctypes.c_void_p(0x900000)
+    for f in fields:
+        p = mep._PlanStruct(**aligned)
+        setattr(p, f, aligned[f] + 2)           # off every alignment the plan needs
+        assert L.mep_plan_noalloc(s, idx, ctypes.byref(p), None) == 2, f
+        p = mep._PlanStruct(**aligned)
+        setattr(p, f, None)
+        assert L.mep_plan_noalloc(s, idx, ctypes.byref(p), None) == 1, f
+    p = mep._PlanStruct(**aligned)
+    assert L.mep_plan_noalloc(s, ctypes.c_void_p(0x900002), ctypes.byref(p), None) == 2
+
+
 def _host_fields(plan):
     h = plan.host()
     ns, nr = h["num_seg"], h["num_replicas"]

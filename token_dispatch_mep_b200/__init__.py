@@ -19,6 +19,7 @@ import torch
 __all__ = [
     "MepError", "Shape", "Plan", "load_library", "library_path",
     "mep_plan_workspace_bytes", "mep_maxvio", "mep_plan", "mep_plan_home_first", "mep_plan_noalloc",
+    "mep_plan_capped", "mep_rank_histogram", "mep_plan_rank", "SCHEDULES", "mep_rank_barrier",
     "mep_dispatch",
     "mep_combine", "mep_combine_backward", "mep_dispatch_backward", "mep_prefetch_replica_weights",
     "mep_dispatch_ranked", "mep_combine_ranked", "rank_pointer_table", "pointer_table",
@@ -42,7 +43,8 @@ ABI_SYMBOLS = ("mep_plan_workspace_bytes", "mep_maxvio", "mep_plan", "mep_dispat
                "mep_prefetch_replica_weights", "mep_plan_home_first", "mep_dispatch_ranked",
                "mep_combine_ranked", "mep_dispatch_ranked_tokens", "mep_combine_ranked_tokens",
                "mep_reduce_replica_grads_ranked", "mep_ipc_export", "mep_ipc_open",
-               "mep_ipc_close")
+               "mep_ipc_close", "mep_plan_capped", "mep_rank_histogram", "mep_plan_rank",
+               "mep_rank_barrier")
 
 
 class MepError(RuntimeError):
@@ -126,6 +128,10 @@ def load_library():
         "mep_dispatch_backward": ([Shape, i32, P, vp, vp, vp], ctypes.c_int),
         "mep_prefetch_replica_weights": ([Shape, P, i64, vp, vp, vp], ctypes.c_int),
         "mep_plan_home_first": ([Shape, vp, P, vp, sz, vp], ctypes.c_int),
+        "mep_plan_capped": ([Shape, i32, vp, P, vp, vp, sz, vp], ctypes.c_int),
+        "mep_rank_histogram": ([Shape, vp, vp, vp, vp, sz, vp], ctypes.c_int),
+        "mep_plan_rank": ([Shape, i32, i32, i32, vp, vp, P, vp, vp, sz, vp], ctypes.c_int),
+        "mep_rank_barrier": ([vp, vp, i32, i32, ctypes.c_uint32, vp, vp], ctypes.c_int),
         "mep_dispatch_ranked": ([Shape, i32, P, vp, vp, vp], ctypes.c_int),
         "mep_combine_ranked": ([Shape, i32, P, vp, vp, vp, vp], ctypes.c_int),
         "mep_dispatch_ranked_tokens": ([Shape, i32, P, i64, i64, vp, vp, vp], ctypes.c_int),
@@ -266,6 +272,90 @@ def mep_plan_home_first(shape, topk_idx, plan: Plan, workspace=None):
     ws = _need(ws_t, "workspace", torch.uint8, mep_plan_workspace_bytes(s), dev)
     _ok(L.mep_plan_home_first(s, idx, ctypes.byref(plan.struct), ws, ws_t.numel(), _stream(dev)),
         "mep_plan_home_first")
+
+
+def mep_plan_capped(shape, B: int, topk_idx, plan: Plan, max_rank_replicas=None, workspace=None):
+    """The capped plan of ``topk_idx`` into ``plan``: at most ``B`` replica
+    experts per rank when every filler finds a room (always when ``B >= 3``
+    and the overflow is large next to the rooms; see ``include/mep.h``).
+    ``max_rank_replicas`` (int32 [1] on the device; default: a new tensor)
+    receives the most replica segments on one rank and is returned."""
+    L, s = load_library(), _shape(shape)
+    dev = plan.device
+    idx = _need(topk_idx, "topk_idx", torch.int32, s.NK, dev)
+    if max_rank_replicas is None:
+        max_rank_replicas = torch.zeros(1, dtype=torch.int32, device=dev)
+    mr = _need(max_rank_replicas, "max_rank_replicas", torch.int32, 1, dev)
+    ws_t = plan.workspace if workspace is None else workspace
+    ws = _need(ws_t, "workspace", torch.uint8, mep_plan_workspace_bytes(s), dev)
+    _ok(L.mep_plan_capped(s, int(B), idx, ctypes.byref(plan.struct), mr, ws, ws_t.numel(),
+                          _stream(dev)), "mep_plan_capped")
+    return max_rank_replicas
+
+
+# mep_schedule_t
+SCHEDULES = {"contiguous": 0, "home_first": 1, "capped": 2}
+
+
+def mep_rank_histogram(shape, local_idx, counts=None, plan: Plan = None, workspace=None):
+    """One rank's histogram: ``counts[e]`` = pairs of ``local_idx`` (int32
+    [S, K]) routed to expert e.  ``workspace``/``plan`` supply the workspace
+    and status word (default: ``plan``'s).  Returns ``counts`` (int32 [E])."""
+    L, s = load_library(), _shape(shape)
+    dev = local_idx.device
+    if counts is None:
+        counts = torch.zeros(s.E, dtype=torch.int32, device=dev)
+    if plan is None:
+        raise ValueError("mep_rank_histogram needs a Plan (workspace and status word)")
+    li = _need(local_idx, "local_idx", torch.int32, s.SK, dev)
+    cp = _need(counts, "counts", torch.int32, s.E, dev)
+    ws_t = plan.workspace if workspace is None else workspace
+    ws = _need(ws_t, "workspace", torch.uint8, mep_plan_workspace_bytes(s), dev)
+    st = ctypes.c_void_p(plan.status_tensor.data_ptr())
+    _ok(L.mep_rank_histogram(s, li, cp, st, ws, ws_t.numel(), _stream(dev)), "mep_rank_histogram")
+    return counts
+
+
+def mep_plan_rank(shape, schedule: str, rank: int, local_idx, rank_counts, plan: Plan, B: int = 0,
+                  max_rank_replicas=None, workspace=None):
+    """Rank ``rank``'s share of the plan from the gathered histograms
+    ``rank_counts`` (int32 [R, E]): every table of the whole-range plan of
+    ``schedule`` ("contiguous", "home_first" or "capped"), and the slots of
+    the rank's own pairs (``local_idx``, int32 [S, K]).  Returns
+    ``max_rank_replicas`` for the capped schedule (else None)."""
+    L, s = load_library(), _shape(shape)
+    dev = plan.device
+    if schedule not in SCHEDULES:
+        raise ValueError(f"unknown schedule {schedule!r}")
+    li = _need(local_idx, "local_idx", torch.int32, s.SK, dev)
+    rc = _need(rank_counts, "rank_counts", torch.int32, s.R * s.E, dev)
+    mr = None
+    if schedule == "capped":
+        if max_rank_replicas is None:
+            max_rank_replicas = torch.zeros(1, dtype=torch.int32, device=dev)
+        mr = _need(max_rank_replicas, "max_rank_replicas", torch.int32, 1, dev)
+    ws_t = plan.workspace if workspace is None else workspace
+    ws = _need(ws_t, "workspace", torch.uint8, mep_plan_workspace_bytes(s), dev)
+    _ok(L.mep_plan_rank(s, SCHEDULES[schedule], int(B), int(rank), li, rc, ctypes.byref(plan.struct),
+                        mr, ws, ws_t.numel(), _stream(dev)), "mep_plan_rank")
+    return max_rank_replicas if schedule == "capped" else None
+
+
+def mep_rank_barrier(peer_flags, my_flags, rank: int, epoch: int, status):
+    """The device barrier between R ranks (``include/mep.h``): ``peer_flags``
+    int64 [R] device array of the ranks' flag-array addresses, ``my_flags``
+    uint32-sized words of this rank (an int32 [R] tensor), ``status`` int32
+    [1] on the device.  Runs on the current stream of ``my_flags``' device
+    (or of ``status``' device when the flags live in host memory)."""
+    L = load_library()
+    dev = status.device
+    R = int(my_flags.numel())
+    tp = _need(peer_flags, "peer_flags", torch.int64, R, peer_flags.device)
+    if my_flags.dtype != torch.int32 or not my_flags.is_contiguous():
+        raise TypeError("my_flags must be a contiguous int32 tensor")
+    sp = _need(status, "status", torch.int32, 1, dev)
+    _ok(L.mep_rank_barrier(tp, ctypes.c_void_p(my_flags.data_ptr()), R, int(rank),
+                           int(epoch) & 0xFFFFFFFF, sp, _stream(dev)), "mep_rank_barrier")
 
 
 def mep_plan_noalloc(shape, topk_idx, plan: Plan):

@@ -48,6 +48,29 @@ cudaStream_t as_stream(void *s) { return static_cast<cudaStream_t>(s); }
 
 }  // namespace
 
+namespace mep {
+
+mep_status_t check_plan_args(const mep_shape_t &shape, const int32_t *topk_idx,
+                             const mep_plan_t *plan) {
+  mep_status_t st = check_shape(shape);
+  if (st != MEP_OK) return st;
+  if (!topk_idx || !plan) return MEP_ERR_INVALID_ARG;
+  const mep_plan_t &p = *plan;
+  if (!p.counts || !p.expert_offset || !p.slot || !p.src_pair || !p.seg || !p.rank_seg_ptr ||
+      !p.expert_seg_ptr || !p.replica_seg || !p.num_seg || !p.num_replicas || !p.max_count ||
+      !p.status || !p.maxvio || !p.rank_seg_idx)
+    return MEP_ERR_INVALID_ARG;
+  const void *i32s[] = {topk_idx, p.counts, p.expert_offset, p.slot, p.src_pair, p.rank_seg_ptr,
+                        p.expert_seg_ptr, p.replica_seg, p.num_seg, p.num_replicas,
+                        p.max_count, p.status, p.rank_seg_idx};
+  for (const void *q : i32s)
+    if (!aligned(q, 4)) return MEP_ERR_MISALIGNED;
+  if (!aligned(p.seg, 16) || !aligned(p.maxvio, 8)) return MEP_ERR_MISALIGNED;
+  return MEP_OK;
+}
+
+}  // namespace mep
+
 extern "C" {
 
 size_t mep_plan_workspace_bytes(mep_shape_t shape) {
@@ -78,22 +101,10 @@ namespace {
 
 mep_status_t plan_common(mep_shape_t shape, const int32_t *topk_idx, const mep_plan_t *plan,
                          void *ws, size_t ws_bytes, void *stream, int kind) {
-  mep_status_t st = check_shape(shape);
+  mep_status_t st = mep::check_plan_args(shape, topk_idx, plan);
   if (st != MEP_OK) return st;
-  if (!topk_idx || !plan) return MEP_ERR_INVALID_ARG;
-  const mep_plan_t &p = *plan;
-  if (!p.counts || !p.expert_offset || !p.slot || !p.src_pair || !p.seg || !p.rank_seg_ptr ||
-      !p.expert_seg_ptr || !p.replica_seg || !p.num_seg || !p.num_replicas || !p.max_count ||
-      !p.status || !p.maxvio || !p.rank_seg_idx)
-    return MEP_ERR_INVALID_ARG;
-  const void *i32s[] = {topk_idx, p.counts, p.expert_offset, p.slot, p.src_pair, p.rank_seg_ptr,
-                        p.expert_seg_ptr, p.replica_seg, p.num_seg, p.num_replicas,
-                        p.max_count, p.status, p.rank_seg_idx};
-  for (const void *q : i32s)
-    if (!aligned(q, 4)) return MEP_ERR_MISALIGNED;
-  if (!aligned(p.seg, 16) || !aligned(p.maxvio, 8)) return MEP_ERR_MISALIGNED;
   if ((st = check_ws(shape, ws, ws_bytes)) != MEP_OK) return st;
-  return from_cuda(mep::launch_plan(shape, topk_idx, p, 1, kind, ws, g_wait_ns.load(), as_stream(stream)));
+  return from_cuda(mep::launch_plan(shape, topk_idx, *plan, 1, kind, ws, g_wait_ns.load(), as_stream(stream)));
 }
 
 }  // namespace
@@ -106,6 +117,68 @@ mep_status_t mep_plan(mep_shape_t shape, const int32_t *topk_idx, const mep_plan
 mep_status_t mep_plan_home_first(mep_shape_t shape, const int32_t *topk_idx,
                                  const mep_plan_t *plan, void *ws, size_t ws_bytes, void *stream) {
   return plan_common(shape, topk_idx, plan, ws, ws_bytes, stream, mep::kPlanHomeFirst);
+}
+
+mep_status_t mep_plan_capped(mep_shape_t shape, int32_t B, const int32_t *topk_idx,
+                             const mep_plan_t *plan, int32_t *max_rank_replicas, void *ws,
+                             size_t ws_bytes, void *stream) {
+  mep_status_t st = mep::check_plan_args(shape, topk_idx, plan);
+  if (st != MEP_OK) return st;
+  if (B < 1 || !max_rank_replicas) return MEP_ERR_INVALID_ARG;
+  if (!aligned(max_rank_replicas, 4)) return MEP_ERR_MISALIGNED;
+  if ((st = check_ws(shape, ws, ws_bytes)) != MEP_OK) return st;
+  // rounds of fillers beyond E can never be used: keep B - 2 in range
+  mep::PlanExtra x;
+  x.B = B > shape.E + 2 ? shape.E + 2 : B;
+  x.max_rank_replicas = max_rank_replicas;
+  return from_cuda(mep::launch_plan(shape, topk_idx, *plan, 1, mep::kPlanCapped, ws,
+                                    g_wait_ns.load(), as_stream(stream), &x));
+}
+
+mep_status_t mep_rank_histogram(mep_shape_t shape, const int32_t *local_idx, int32_t *counts,
+                                int32_t *status, void *ws, size_t ws_bytes, void *stream) {
+  mep_status_t st = check_shape(shape);
+  if (st != MEP_OK) return st;
+  if (!local_idx || !counts || !status) return MEP_ERR_INVALID_ARG;
+  if (!aligned(local_idx, 4) || !aligned(counts, 4) || !aligned(status, 4))
+    return MEP_ERR_MISALIGNED;
+  if ((st = check_ws(shape, ws, ws_bytes)) != MEP_OK) return st;
+  // the histogram of one rank's S*K pairs: the counting pass over a
+  // one-rank shape (max_count and maxvio are not wanted)
+  const mep_shape_t one{1, shape.S, shape.E, shape.K};
+  mep_plan_t pl{};
+  pl.counts = counts;
+  pl.status = status;
+  return from_cuda(mep::launch_plan(one, local_idx, pl, 0, mep::kPlanContiguous, ws,
+                                    g_wait_ns.load(), as_stream(stream)));
+}
+
+mep_status_t mep_plan_rank(mep_shape_t shape, int32_t schedule, int32_t B, int32_t rank,
+                           const int32_t *local_idx, const int32_t *rank_counts,
+                           const mep_plan_t *plan, int32_t *max_rank_replicas, void *ws,
+                           size_t ws_bytes, void *stream) {
+  mep_status_t st = mep::check_plan_args(shape, local_idx, plan);
+  if (st != MEP_OK) return st;
+  if (rank < 0 || rank >= shape.R || !rank_counts) return MEP_ERR_INVALID_ARG;
+  if (schedule != MEP_SCHEDULE_CONTIGUOUS && schedule != MEP_SCHEDULE_HOME_FIRST &&
+      schedule != MEP_SCHEDULE_CAPPED)
+    return MEP_ERR_INVALID_ARG;
+  if (schedule == MEP_SCHEDULE_CAPPED && (B < 1 || !max_rank_replicas)) return MEP_ERR_INVALID_ARG;
+  if (!aligned(rank_counts, 4) || (max_rank_replicas && !aligned(max_rank_replicas, 4)))
+    return MEP_ERR_MISALIGNED;
+  if ((st = check_ws(shape, ws, ws_bytes)) != MEP_OK) return st;
+  mep::PlanExtra x;
+  x.rank_counts = rank_counts;
+  x.rank = rank;
+  int kind = mep::kPlanContiguous;
+  if (schedule == MEP_SCHEDULE_HOME_FIRST) kind = mep::kPlanHomeFirst;
+  if (schedule == MEP_SCHEDULE_CAPPED) {
+    kind = mep::kPlanCapped;
+    x.B = B > shape.E + 2 ? shape.E + 2 : B;
+    x.max_rank_replicas = max_rank_replicas;
+  }
+  return from_cuda(mep::launch_plan(shape, local_idx, *plan, 1, kind, ws, g_wait_ns.load(),
+                                    as_stream(stream), &x));
 }
 
 mep_status_t mep_dispatch(mep_shape_t shape, int32_t H, const mep_plan_t *plan, const uint16_t *x,
@@ -265,6 +338,16 @@ mep_status_t mep_reduce_replica_grads_ranked(mep_shape_t shape, const mep_plan_t
     return MEP_ERR_MISALIGNED;
   return from_cuda(mep::launch_reduce_ranked(shape, *plan, P, home_rank, rank_grads, rank_rows,
                                              home_grads, as_stream(stream)));
+}
+
+mep_status_t mep_rank_barrier(uint32_t *const *peer_flags, uint32_t *my_flags, int32_t R,
+                              int32_t rank, uint32_t epoch, int32_t *status, void *stream) {
+  if (R < 1 || R > MEP_MAX_RANKS || rank < 0 || rank >= R) return MEP_ERR_INVALID_ARG;
+  if (!peer_flags || !my_flags || !status) return MEP_ERR_INVALID_ARG;
+  if (!aligned(peer_flags, 8) || !aligned(my_flags, 4) || !aligned(status, 4))
+    return MEP_ERR_MISALIGNED;
+  return from_cuda(mep::launch_rank_barrier(peer_flags, my_flags, R, rank, epoch, status,
+                                            g_wait_ns.load(), as_stream(stream)));
 }
 
 mep_status_t mep_read_status(const mep_plan_t *plan, void *stream) {

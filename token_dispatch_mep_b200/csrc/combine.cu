@@ -1,22 +1,42 @@
 // Weighted combine back to token order:
 //   out[g, :] = bf16_rne( sum_{k=0..K-1} w[g,k] * y[slot[g,k], :] )
-// accumulated in float32 with one fused multiply-add per term, k ascending.
+// with the K terms added in binary64, k ascending, and the sum rounded once.
 //
 // Method: a router assigns every token to K experts (MoonEP release page,
 // "Why expert parallelism is needed"); the K expert outputs return to the
 // token's position, weighted by the router weights.
 //
+// Arithmetic.  A float32 weight times a bf16 value has at most 24 + 8
+// significant bits, so every product is exact in binary64, and a chain of
+// binary64 fused multiply-adds in k order, acc = fma(w_k, y_k, acc), rounds
+// exactly like adding the exact products one by one.  The sum is then
+// rounded once to bf16 (round to nearest, ties to even), so the result is the
+// correctly rounded value of the k-ordered binary64 sum -- whatever the
+// cancellation between terms.  A float32 accumulator could not promise that:
+// under cancellation its rounding errors can move the result by several bf16
+// units.  The kernel stays bound by HBM bandwidth: about five integer or FP64
+// instructions per 2-byte element read.
+//   bf16 -> binary64 without a conversion instruction: the bf16 bits b placed
+//   as the top of a binary64 word -- sign to bit 63, the 8 exponent bits to
+//   the low end of the 11-bit exponent field, the 7 fraction bits to the top
+//   of the fraction -- give exactly y * 2^-896 for every finite y (zero and
+//   subnormals included: the two formats' subnormal scales differ by the same
+//   2^-896), and the weight is scaled by 2^896 once per term (exact: a float32
+//   times 2^896 stays below 2^1024).  Infinities and NaNs do not survive this
+//   mapping, so every loaded word is checked for an all-ones exponent; a chunk
+//   that holds one is summed again with exact conversions (the oracle's
+//   arithmetic: inf and NaN propagate).
+//
 // One warp per token walks the row, kRU = 2 16-byte chunks (8 bf16 each) per
 // lane per step.  Lanes k < K hold the token's slot id and weight, which the
 // warp broadcasts with shuffles.  The K expert-output chunks are loaded in
-// groups of 8 (all loads of a group issued before any use) and added in k
-// order with one float32 FMA each, so every output is the same k-ordered
-// float32 sum whatever the grouping; the sum is rounded to bf16 and written
-// with a streaming 16-byte store.  Expert outputs are read once (streaming
-// loads).  The grid has one warp per token, in blocks of two warps: small
-// blocks keep the last wave short (1 % over blocks of eight warps).  A form
-// with warp tasks over parts of rows and all K loads in flight measured
-// 0.90-1.00 of the HBM copy peak against 0.96-1.04 for this one.
+// groups of 8 (all loads of a group issued before any use) and accumulated in
+// k order; the sum is rounded to bf16 and written with a streaming 16-byte
+// store.  Expert outputs are read once (streaming loads).  The grid has one
+// warp per token, in blocks of two warps: small blocks keep the last wave
+// short (1 % over blocks of eight warps).  A form with warp tasks over parts
+// of rows and all K loads in flight measured 0.90-1.00 of the HBM copy peak
+// against 0.96-1.04 for this one.
 //
 // Rank-addressed form (mep_combine_ranked): expert outputs are read from R
 // separate rank buffers, slot p being row p % SK of rank_ys[p / SK]; a NULL
@@ -25,8 +45,8 @@
 // range's; mep_combine_ranked_tokens).
 //
 // With no weights (w == nullptr) every weight is 1 and the kernel is the
-// backward of dispatch: grad_x[g] = bf16(sum_k grad_buf[slot[g,k]]) (an FMA
-// with weight 1 rounds exactly like an addition).
+// backward of dispatch: grad_x[g] = bf16(sum_k grad_buf[slot[g,k]]), the same
+// binary64 sum rounded once.
 #include <algorithm>
 #include <cstdint>
 
@@ -40,6 +60,12 @@
 #endif
 #ifndef MEP_COMBINE_ROW_U
 #define MEP_COMBINE_ROW_U 2  // 16-byte chunks per lane per step
+#endif
+#ifndef MEP_COMBINE_NF_MAX
+#define MEP_COMBINE_NF_MAX 0  // 1: non-finite check by a 16x2 max of the exponents
+#endif
+#ifndef MEP_COMBINE_CVT
+#define MEP_COMBINE_CVT 0  // 1: bf16 -> float32 -> binary64 by conversion instructions
 #endif
 
 namespace mep {
@@ -63,25 +89,105 @@ struct CombineParams {
   int32_t chunks;      // 16-byte chunks per row = H / 8
 };
 
-__device__ __forceinline__ void fma8(float (&acc)[8], float wk, const uint4 &v) {
+constexpr double kTwo896 = 0x1p896;  // scale of the integer bf16 -> binary64 mapping
+
+// Binary64 word whose value is y * 2^-896 for the bf16 y held in the top half
+// of `x` (the low 16 bits of x are ignored): the sign stays at bit 31 of the
+// high word, the arithmetic shift moves the exponent to bits 20..27 and the
+// fraction to bits 13..19, and the mask clears the sign copies in bits 28..30
+// and the low bits.
+__device__ __forceinline__ double bf16_hi_to_scaled_f64(uint32_t x) {
+  return __hiloint2double((int)(((int32_t)x >> 3) & (int32_t)0x8fffe000u), 0);
+}
+
+// Nonzero in bit 15 or 31 if a bf16 half of u has an all-ones exponent
+// (infinity or NaN): the masked, inverted exponent of such a half is zero, and
+// subtracting 1 from it sets the half's top bit (no other half value, all
+// multiples of 0x80 below 0x8000, reaches it).
+__device__ __forceinline__ uint32_t nonfinite_bits(uint32_t u) {
+  return ((~u) & 0x7f807f80u) - 0x00010001u;
+}
+
+#if MEP_COMBINE_NF_MAX
+__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+#endif
+
+// acc[j] = fma(ws, y_j * 2^-896, acc[j]) for the 8 bf16 of v (ws = w * 2^896),
+// in element order; *nf collects the non-finite check of the loaded words.
+__device__ __forceinline__ void fma8(double (&acc)[8], double ws, const uint4 &v, uint32_t *nf) {
   const uint32_t u[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    const float lo = __uint_as_float(u[j] << 16);
-    const float hi = __uint_as_float(u[j] & 0xffff0000u);
-    acc[2 * j] = __fmaf_rn(wk, lo, acc[2 * j]);
-    acc[2 * j + 1] = __fmaf_rn(wk, hi, acc[2 * j + 1]);
+#if MEP_COMBINE_CVT
+    (void)nf;
+    acc[2 * j] = __fma_rn(ws, (double)__uint_as_float(u[j] << 16), acc[2 * j]);
+    acc[2 * j + 1] = __fma_rn(ws, (double)__uint_as_float(u[j] & 0xffff0000u), acc[2 * j + 1]);
+#else
+#if MEP_COMBINE_NF_MAX
+    *nf = max_u16x2(*nf, u[j] & 0x7f807f80u);
+#else
+    *nf |= nonfinite_bits(u[j]);
+#endif
+    acc[2 * j] = __fma_rn(ws, bf16_hi_to_scaled_f64(u[j] << 16), acc[2 * j]);
+    acc[2 * j + 1] = __fma_rn(ws, bf16_hi_to_scaled_f64(u[j]), acc[2 * j + 1]);
+#endif
   }
 }
 
-__device__ __forceinline__ uint4 pack8(const float (&acc)[8]) {
+// Nonzero if the collected check saw an infinity or NaN.
+__device__ __forceinline__ bool saw_nonfinite(uint32_t nf) {
+#if MEP_COMBINE_CVT
+  (void)nf;
+  return false;
+#elif MEP_COMBINE_NF_MAX
+  return (nf & 0xffffu) == 0x7f80u || (nf >> 16) == 0x7f80u;
+#else
+  return (nf & 0x80008000u) != 0;
+#endif
+}
+
+// The same sum with exact conversions (no scaling): infinities and NaNs
+// propagate as in binary64 arithmetic.
+__device__ __forceinline__ void fma8_exact(double (&acc)[8], double w, const uint4 &v) {
+  const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    acc[2 * j] = __fma_rn(w, (double)__uint_as_float(u[j] << 16), acc[2 * j]);
+    acc[2 * j + 1] = __fma_rn(w, (double)__uint_as_float(u[j] & 0xffff0000u), acc[2 * j + 1]);
+  }
+}
+
+__device__ __forceinline__ uint4 pack8(const double (&acc)[8]) {
   uint32_t u[4];
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    const __nv_bfloat162 b = __floats2bfloat162_rn(acc[2 * j], acc[2 * j + 1]);
-    u[j] = *reinterpret_cast<const uint32_t *>(&b);
+    const uint32_t lo = __bfloat16_as_ushort(__double2bfloat16(acc[2 * j]));
+    const uint32_t hi = __bfloat16_as_ushort(__double2bfloat16(acc[2 * j + 1]));
+    u[j] = lo | (hi << 16);
   }
   return make_uint4(u[0], u[1], u[2], u[3]);
+}
+
+// Row address of slot pp (ranked form: row pp % SK of rank pp / SK's buffer);
+// clears *ok (and flags *bad if *ok was set) when a rank buffer is missing or
+// misaligned.
+template <bool kRanked>
+__device__ __forceinline__ const uint16_t *slot_row(const CombineParams &p, int64_t pp, bool *ok,
+                                                    bool *bad) {
+  if (kRanked) {
+    const int64_t r = pp / p.SK;
+    const uint16_t *base = p.rank_ys[r];
+    if (base == nullptr || (reinterpret_cast<uintptr_t>(base) & 15) != 0) {
+      if (*ok) *bad = true;
+      *ok = false;
+    }
+    return base + (pp - r * p.SK) * p.H;
+  }
+  return p.y + pp * p.H;
 }
 
 template <int KC, bool kRanked>
@@ -98,14 +204,20 @@ __global__ void __launch_bounds__(kThreads, MEP_COMBINE_MIN_BLOCKS) combine_row_
       bad = true;
       sl = -1;
     }
+#if MEP_COMBINE_CVT
+    const double wts = (double)wt;
+#else
+    const double wts = (double)wt * kTwo896;  // exact
+#endif
     const unsigned okmask = __ballot_sync(0xffffffffu, sl >= 0);
     uint4 *orow = reinterpret_cast<uint4 *>(p.out + g * p.H);
     for (int c0 = 0; c0 < p.chunks; c0 += 32 * kRU) {
-      float acc[kRU][8];
+      double acc[kRU][8];
 #pragma unroll
       for (int u = 0; u < kRU; ++u)
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[u][e] = 0.f;
+        for (int e = 0; e < 8; ++e) acc[u][e] = 0.0;
+      uint32_t nf = 0;
 #pragma unroll
       for (int kg = 0; kg < KC; kg += KG) {
         uint4 v[KG][kRU];
@@ -113,20 +225,7 @@ __global__ void __launch_bounds__(kThreads, MEP_COMBINE_MIN_BLOCKS) combine_row_
         for (int j = 0; j < KG; ++j) {
           const int pk = __shfl_sync(0xffffffffu, sl, kg + j);
           bool ok = ((okmask >> (kg + j)) & 1) && (unsigned)pk < (unsigned)p.NK;
-          const int64_t pp = ok ? pk : 0;
-          const uint16_t *yrow;
-          if (kRanked) {
-            // a rank buffer must be present and 16-byte aligned
-            const int64_t r = pp / p.SK;
-            const uint16_t *base = p.rank_ys[r];
-            if (base == nullptr || (reinterpret_cast<uintptr_t>(base) & 15) != 0) {
-              if (ok) bad = true;
-              ok = false;
-            }
-            yrow = base + (pp - r * p.SK) * p.H;
-          } else {
-            yrow = p.y + pp * p.H;
-          }
+          const uint16_t *yrow = slot_row<kRanked>(p, ok ? pk : 0, &ok, &bad);
 #pragma unroll
           for (int u = 0; u < kRU; ++u) {
             const int c = c0 + u * 32 + lane;
@@ -136,10 +235,34 @@ __global__ void __launch_bounds__(kThreads, MEP_COMBINE_MIN_BLOCKS) combine_row_
         }
 #pragma unroll
         for (int j = 0; j < KG; ++j) {
-          const float wk = __shfl_sync(0xffffffffu, wt, kg + j);
+          const double wk = __shfl_sync(0xffffffffu, wts, kg + j);
           if ((okmask >> (kg + j)) & 1) {
 #pragma unroll
-            for (int u = 0; u < kRU; ++u) fma8(acc[u], wk, v[j][u]);
+            for (int u = 0; u < kRU; ++u) fma8(acc[u], wk, v[j][u], &nf);
+          }
+        }
+      }
+      // A chunk with an infinity or NaN among its inputs: sum it again with
+      // exact conversions (rare; warp-uniform branch, the shuffles need every
+      // lane).
+      const bool redo = saw_nonfinite(nf);
+      if (__any_sync(0xffffffffu, redo)) {
+#pragma unroll
+        for (int u = 0; u < kRU; ++u)
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            if (redo) acc[u][e] = 0.0;
+        for (int k = 0; k < KC; ++k) {
+          const int pk = __shfl_sync(0xffffffffu, sl, k);
+          const double wk = (double)__shfl_sync(0xffffffffu, wt, k);
+          bool ok = redo && k < p.K && ((okmask >> k) & 1) && (unsigned)pk < (unsigned)p.NK;
+          bool ignored = false;
+          const uint16_t *yrow = slot_row<kRanked>(p, ok ? pk : 0, &ok, &ignored);
+#pragma unroll
+          for (int u = 0; u < kRU; ++u) {
+            const int c = c0 + u * 32 + lane;
+            if (ok && c < p.chunks)
+              fma8_exact(acc[u], wk, __ldcs(reinterpret_cast<const uint4 *>(yrow) + c));
           }
         }
       }

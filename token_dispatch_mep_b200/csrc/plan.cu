@@ -74,7 +74,7 @@ struct PlanParams {
   int32_t nt;    // tiles (nb - 1 with a coordinator, else 1)
   int64_t ppb;   // pairs per tile
   int32_t full;  // 0: counts + maxvio only
-  int32_t kind;  // kPlanContiguous or kPlanHomeFirst
+  int32_t kind;  // kPlanContiguous, kPlanHomeFirst or kPlanCapped
   int32_t *counts, *expert_offset, *slot, *src_pair;
   int4 *seg;
   int32_t *rank_seg_ptr, *expert_seg_ptr, *replica_seg, *rank_seg_idx;
@@ -83,6 +83,18 @@ struct PlanParams {
   int32_t *tile;   // workspace [E][nt]
   uint32_t *bar;   // workspace barrier words
   uint64_t wait_ns;
+  // one rank's share (mep_plan_rank): the tiles cover that rank's own pairs,
+  // global pairs [pair0, pair0 + NKt); T_e and the rank prefix come from the
+  // gathered per-rank histograms
+  int64_t pair0;               // global index of the first pair the tiles cover
+  int64_t NKt;                 // pairs the tiles cover (NK for the whole range)
+  const int32_t *rank_counts;  // [R][E] per-rank histograms, or nullptr
+  int32_t rank;                // the rank whose pairs the tiles cover
+  int32_t *totals;             // [E] tile totals of phase 2 (p.counts, or workspace)
+  // capped plan
+  int32_t B;                   // replica experts a rank may host
+  int32_t *max_rank_replicas;  // [1] out
+  int32_t *tab;                // workspace: the scatter tables the coordinator publishes
 };
 
 // Mask of the lanes whose key equals this lane's key; keys are < 2^nbits.
@@ -167,6 +179,385 @@ __device__ __forceinline__ int home_first_slot(int e, int i, int Bx, int C, int 
   return r * C + s_F[r] + (q - s_D[r]);
 }
 
+// Slot of the i-th pair (in (g,k) order) of expert e in the capped plan: the
+// first h_e pairs go home, the others to the piece holding overflow index
+// q = i - h_e (pieces of e in creation order, first overflow indices
+// ascending: a binary search).
+__device__ __forceinline__ int capped_slot(int e, int i, const int *s_h, const int *s_hb,
+                                           const int *s_pb, const int *s_pq, const int *s_pbase) {
+  const int h = s_h[e];
+  if (i < h) return s_hb[e] + i;
+  const int q = i - h;
+  int lo = s_pb[e], hi = s_pb[e + 1];
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (s_pq[mid] <= q) lo = mid; else hi = mid;
+  }
+  return s_pbase[lo] + q;
+}
+
+// Ascending bitonic sort of n keys in shared memory (n a power of two,
+// n <= 2 * blockDim.x); every thread of the block must call it.
+template <typename K>
+__device__ void block_bitonic_sort(K *a, int n) {
+  for (int k = 2; k <= n; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int i = threadIdx.x; i < (n >> 1); i += blockDim.x) {
+        const int lo = ((i & ~(j - 1)) << 1) | (i & (j - 1));
+        const int hi = lo + j;
+        const K x = a[lo], y = a[hi];
+        if ((x > y) == ((lo & k) == 0)) {
+          a[lo] = y;
+          a[hi] = x;
+        }
+      }
+      __syncthreads();
+    }
+  }
+}
+
+// Last index i in [0, n) with a[i] <= x (a nondecreasing, a[0] <= x).
+__device__ __forceinline__ int last_le(const int *a, int n, int x) {
+  return upper_bound_idx(a, n, x) - 1;
+}
+
+// Words of the capped plan's scatter tables in the workspace (published by
+// the coordinator): per expert the pairs kept home h_e, the home slot base
+// and the first of its replica pieces; per piece its first overflow index
+// and its slot base (slot = base + overflow index).
+__host__ __device__ __forceinline__ int64_t capped_tab_words(int E, int R) {
+  return 3 * (int64_t)E + 1 + 2 * ((int64_t)E + R);
+}
+
+// The capped schedule's tables, built by the coordinator block (which owns no
+// pairs, so its dynamic shared memory is free scratch: sm holds at least
+// kWarps * E + kWarps * kPlanIdsPerWarp ints, more than the 18 E + 15 R + 2 n2
+// + 8 (n2 <= 2 (E + R)) this needs, since R <= E <= 1024).  T is this thread's expert count (t < E), s_off
+// the expert offsets.  Writes every plan field except counts, offsets, slot
+// and src_pair, and publishes the scatter tables to p.tab.
+//   1. home fill, smallest home experts first (ties: lower id);
+//   2. items (overflowing experts, overflow descending) and rooms (ranks with
+//      spare room, room descending), in one bitonic sort;
+//   3. fillers (items below the largest room): filler f is offered to room
+//      f mod Y in round f / Y < B - 2, placed whole if it fits -- one thread
+//      per room walks its candidates;
+//   4. the stream: items not placed, cut over the rooms' space left, by
+//      prefix sums and binary searches;
+//   5. the segment table by (expert, rank): a bitonic sort of
+//      (expert, rank, piece) keys.
+__device__ void capped_build(const PlanParams &p, int T, const int *s_off, int *sm, int *s_w) {
+  const int t = threadIdx.x;
+  const int E = p.E, R = p.R, C = (int)p.SK, Bh = E / R;
+  const int NP = E + R;  // bound on replica pieces (at most E + R - 1)
+  int *sT = sm;                 // [E] T_e
+  int *sh = sT + E;             // [E] h_e, pairs kept home
+  int *shb = sh + E;            // [E] home slot base of e
+  int *spb = shb + E;           // [E+1] first replica piece of e
+  int *shl = spb + E + 1;       // [E] index of e's home piece among its rank's segments
+  int *it_e = shl + E;          // [E] expert of item i (step 1: counts in fill order)
+  int *it_O = it_e + E;         // [E] overflow of item i (step 1: scan of those counts)
+  int *it_loc = it_O + E;       // [E] filler: start in its room's replica area, else -1
+  int *it_P = it_loc + E;       // [E+1] stream position of item i (step 1: home prefix)
+  int *it_s = it_P + E + 1;     // [E+1] stream index, or a filler's index in its room
+  int *it_of = it_s + E + 1;    // [E] item index of expert e, -1 if e has no overflow
+  int *st_i = it_of + E;        // [E] item at stream index s
+  int *rm_r = st_i + E;         // [R] rank of room j
+  int *rm_D = rm_r + R;         // [R] spare room
+  int *rm_left = rm_D + R;      // [R] space left after the fillers
+  int *rm_nf = rm_left + R;     // [R] fillers placed
+  int *rm_Q = rm_nf + R;        // [R] stream position of room j's space left
+  int *rm_first = rm_Q + R;     // [R] stream index of the first item meeting room j
+  int *rm_nz = rm_first + R;    // [R+1] rooms with space left before room j
+  int *rk_nh = rm_nz + R + 1;   // [R] home pieces of rank r
+  int *rk_nr = rk_nh + R;       // [R] replica pieces of rank r
+  int *pc_e = rk_nr + R;        // [NP] expert of piece
+  int *pc_r = pc_e + NP;        // [NP] rank of piece
+  int *pc_loc = pc_r + NP;      // [NP] first slot of the piece within its rank
+  int *pc_n = pc_loc + NP;      // [NP] size
+  int *pc_q = pc_n + NP;        // [NP] first overflow index of the piece within its expert
+  int *pc_li = pc_q + NP;       // [NP] index among its rank's segments (slot order)
+  uint64_t *keys = reinterpret_cast<uint64_t *>(
+      (reinterpret_cast<uintptr_t>(pc_li + NP) + 7) & ~static_cast<uintptr_t>(7));  // [n2]
+  uint32_t *skeys = reinterpret_cast<uint32_t *>(keys);  // step 5 reuses the key buffer
+  int tot;
+
+  // ---- 1. home fill, smallest home experts first --------------------------
+  if (t < E) sT[t] = T;
+  __syncthreads();
+  const int b0 = t < E ? (t / Bh) * Bh : 0;
+  int pos = t;  // position of e in (home block, count, id) order
+  if (t < E && R > 1) {
+    int rk = 0;
+    for (int e2 = b0; e2 < b0 + Bh; ++e2) {
+      const int v = sT[e2];
+      rk += (v < T || (v == T && e2 < t)) ? 1 : 0;
+    }
+    pos = b0 + rk;
+  }
+  if (t < E) it_e[pos] = T;
+  __syncthreads();
+  const int fx = block_excl_scan(t < E ? it_e[t] : 0, &tot, s_w);
+  if (t < E) it_O[t] = fx;
+  __syncthreads();
+  // with one rank every pair fits at home
+  const int h = t < E ? (R == 1 ? T : max(0, min(T, C - (it_O[pos] - it_O[b0])))) : 0;
+  const int O = t < E ? T - h : 0;
+  int hf_tot;
+  const int hx = block_excl_scan(h, &tot, s_w);                  // home prefix, expert order
+  const int hf = block_excl_scan(h > 0 ? 1 : 0, &hf_tot, s_w);  // home pieces before e
+  if (t < E) {
+    it_P[t] = hx;
+    it_s[t] = hf;
+  }
+  if (t == 0) it_s[E] = hf_tot;
+  __syncthreads();
+  if (t < E) {
+    sh[t] = h;
+    shb[t] = (t / Bh) * C + (hx - it_P[b0]);
+    shl[t] = hf - it_s[b0];
+  }
+  if (t < R) rk_nh[t] = it_s[(t + 1) * Bh] - it_s[t * Bh];
+  // spare room of rank t: its home load is s_off over its block
+  const int Dr = t < R ? C - min(s_off[(t + 1) * Bh] - s_off[t * Bh], C) : 0;
+
+  // ---- 2. items and rooms in one sort -------------------------------------
+  int n2 = 2;
+  while (n2 < E + R) n2 <<= 1;
+  const int X = __syncthreads_count(t < E && O > 0);
+  const int Y = __syncthreads_count(t < R && Dr > 0);
+  for (int i = t; i < n2; i += kThreads) {
+    uint64_t k = ~0ull;
+    if (i < E) {
+      const int Oi = sT[i] - sh[i];
+      if (Oi > 0) k = ((uint64_t)(0x7fffffff - Oi) << 32) | (uint32_t)i;
+    } else if (i < E + R) {
+      const int r = i - E;
+      const int Dx = C - min(s_off[(r + 1) * Bh] - s_off[r * Bh], C);
+      if (Dx > 0) k = (1ull << 63) | ((uint64_t)(0x7fffffff - Dx) << 32) | (uint32_t)r;
+    }
+    keys[i] = k;
+  }
+  __syncthreads();
+  block_bitonic_sort(keys, n2);
+  if (t < E) it_of[t] = -1;
+  __syncthreads();
+  if (t < X) {
+    const uint64_t k = keys[t];
+    const int e = (int)(k & 0xffffffffu);
+    it_e[t] = e;
+    it_O[t] = 0x7fffffff - (int)((k >> 32) & 0x7fffffff);
+    it_of[e] = t;
+    it_loc[t] = -1;
+  }
+  if (t < Y) {
+    const uint64_t k = keys[X + t];
+    rm_r[t] = (int)(k & 0xffffffffu);
+    rm_D[t] = 0x7fffffff - (int)((k >> 32) & 0x7fffffff);
+  }
+  __syncthreads();
+
+  // ---- 3. fillers ----------------------------------------------------------
+  const int dmax = Y > 0 ? rm_D[0] : 0;
+  const int i0 = __syncthreads_count(t < X && it_O[t] >= dmax);  // items at least dmax
+  const int nf = X - i0;
+  if (t < Y) {
+    int left = rm_D[t], cnt = 0;
+    for (int round = 0; round < p.B - 2; ++round) {
+      const int f = t + round * Y;
+      if (f >= nf) break;
+      const int i = i0 + f;
+      if (it_O[i] <= left) {
+        it_loc[i] = rm_D[t] - left;
+        it_s[i] = cnt;  // index among the room's fillers
+        left -= it_O[i];
+        ++cnt;
+      }
+    }
+    rm_left[t] = left;
+    rm_nf[t] = cnt;
+  }
+  __syncthreads();
+
+  // ---- 4. the stream -------------------------------------------------------
+  const bool ins = t < X && it_loc[t] < 0;
+  int ns_items;
+  const int P = block_excl_scan(ins ? it_O[t] : 0, &tot, s_w);
+  const int si = block_excl_scan(ins ? 1 : 0, &ns_items, s_w);
+  const int Q = block_excl_scan(t < Y ? rm_left[t] : 0, &tot, s_w);
+  const int nzx = block_excl_scan(t < Y && rm_left[t] > 0 ? 1 : 0, &tot, s_w);
+  if (ins) {
+    it_P[t] = P;
+    it_s[t] = si;
+    st_i[si] = t;
+  }
+  if (t < Y) {
+    rm_Q[t] = Q;
+    rm_nz[t] = nzx;
+  }
+  if (t == 0) rm_nz[Y] = tot;
+  __syncthreads();
+  // stream index of the first item meeting room j
+  if (t < Y && rm_left[t] > 0) {
+    int lo = 0, hi = ns_items;  // last s with P(st_i[s]) <= Q
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (it_P[st_i[mid]] <= rm_Q[t]) lo = mid; else hi = mid;
+    }
+    rm_first[t] = lo;
+  }
+  __syncthreads();
+  // pieces of expert t: its filler, or its stream pieces
+  int npc = 0, j0 = 0, j1 = -1;
+  const int it = t < E ? it_of[t] : -1;
+  if (it >= 0) {
+    if (it_loc[it] >= 0) {
+      npc = 1;
+    } else {
+      const int a = it_P[it], b = a + it_O[it];
+      j0 = last_le(rm_Q, Y, a);
+      j1 = last_le(rm_Q, Y, b - 1);
+      npc = rm_nz[j1 + 1] - rm_nz[j0];
+    }
+  }
+  int npieces;
+  const int pb = block_excl_scan(npc, &npieces, s_w);
+  if (t < E) spb[t] = pb;
+  if (t == 0) spb[E] = npieces;
+  __syncthreads();
+  if (it >= 0 && pb + npc <= NP) {  // at most E + R - 1 pieces by construction
+    const int e = t;
+    if (it_loc[it] >= 0) {
+      const int j = (it - i0) % Y;
+      const int r = rm_r[j];
+      pc_e[pb] = e;
+      pc_r[pb] = r;
+      pc_loc[pb] = (C - rm_D[j]) + it_loc[it];
+      pc_n[pb] = it_O[it];
+      pc_q[pb] = 0;
+      pc_li[pb] = rk_nh[r] + it_s[it];
+    } else {
+      const int a = it_P[it], b = a + it_O[it];
+      int q = pb;
+      for (int j = j0; j <= j1; ++j) {
+        if (rm_left[j] == 0) continue;
+        const int r = rm_r[j];
+        const int lo = max(a, rm_Q[j]), hi = min(b, rm_Q[j] + rm_left[j]);
+        pc_e[q] = e;
+        pc_r[q] = r;
+        pc_loc[q] = (C - rm_D[j]) + (rm_D[j] - rm_left[j]) + (lo - rm_Q[j]);
+        pc_n[q] = hi - lo;
+        pc_q[q] = lo - a;
+        pc_li[q] = rk_nh[r] + rm_nf[j] + (it_s[it] - rm_first[j]);
+        ++q;
+      }
+    }
+  }
+  // replica pieces per rank: fillers plus the stream items meeting the room
+  if (t < R) rk_nr[t] = 0;
+  __syncthreads();
+  int nrep_j = 0;
+  if (t < Y) {
+    int nst = 0;
+    if (rm_left[t] > 0) {
+      int lo = 0, hi = ns_items;  // last s with P(st_i[s]) <= Q + left - 1
+      const int last = rm_Q[t] + rm_left[t] - 1;
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (it_P[st_i[mid]] <= last) lo = mid; else hi = mid;
+      }
+      nst = lo - rm_first[t] + 1;
+    }
+    nrep_j = rm_nf[t] + nst;
+    rk_nr[rm_r[t]] = nrep_j;
+  }
+  const int mx = block_max(nrep_j, s_w);  // syncs
+  // publish the scatter tables
+  int *tab_h = p.tab, *tab_hb = tab_h + E, *tab_pb = tab_hb + E;
+  int *tab_pq = tab_pb + E + 1, *tab_pbase = tab_pq + NP;
+  if (t < E) {
+    __stcg(tab_h + t, sh[t]);
+    __stcg(tab_hb + t, shb[t]);
+    __stcg(tab_pb + t, spb[t]);
+  }
+  if (t == 0) __stcg(tab_pb + E, spb[E]);
+  for (int q = t; q < npieces; q += kThreads) {
+    __stcg(tab_pq + q, pc_q[q]);
+    __stcg(tab_pbase + q, pc_r[q] * C + pc_loc[q] - pc_q[q]);
+  }
+
+  // ---- 5. the segment table, by (expert, rank) -----------------------------
+  const int nhome = it_s[E];
+  const int nseg = nhome + npieces;
+  int m2 = 2;
+  while (m2 < nseg) m2 <<= 1;
+  // keys: expert (bits 21..30), rank (11..20), piece id (0..10; 2047 = home)
+  for (int i = t; i < m2; i += kThreads) skeys[i] = 0xffffffffu;
+  __syncthreads();
+  if (t < E && h > 0) skeys[hf] = ((uint32_t)t << 21) | ((uint32_t)(t / Bh) << 11) | 2047u;
+  for (int q = t; q < npieces; q += kThreads)
+    skeys[nhome + q] = ((uint32_t)pc_e[q] << 21) | ((uint32_t)pc_r[q] << 11) | (uint32_t)q;
+  __syncthreads();
+  block_bitonic_sort(skeys, m2);
+  // rank_seg_ptr: each rank's home and replica segments
+  int rtot;
+  const int rsp = block_excl_scan(t < R ? rk_nh[t] + rk_nr[t] : 0, &rtot, s_w);
+  if (t < R) {
+    p.rank_seg_ptr[t] = rsp;
+    rm_Q[t] = rsp;  // rank_seg_ptr, kept for the writes below (rm_Q is no longer needed)
+  }
+  if (t == 0) p.rank_seg_ptr[R] = rtot;
+  __syncthreads();
+  // segments a = 2t and 2t + 1 of the table (at most 2047 of them)
+  bool rep[2];
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int a = 2 * t + u;
+    rep[u] = false;
+    if (a < nseg) {
+      const uint32_t k = skeys[a];
+      rep[u] = (int)((k >> 11) & 1023u) != (int)(k >> 21) / Bh;
+    }
+  }
+  int nrep_tot;
+  int rpos = block_excl_scan((rep[0] ? 1 : 0) + (rep[1] ? 1 : 0), &nrep_tot, s_w);
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int a = 2 * t + u;
+    if (a >= nseg) continue;
+    const uint32_t k = skeys[a];
+    const int e = (int)(k >> 21), r = (int)((k >> 11) & 1023u), pid = (int)(k & 2047u);
+    int start, cnt, li;
+    if (pid == 2047) {
+      start = shb[e] - r * C;
+      cnt = sh[e];
+      li = shl[e];
+    } else {
+      start = pc_loc[pid];
+      cnt = pc_n[pid];
+      li = pc_li[pid];
+    }
+    p.seg[a] = make_int4(e, r, start, cnt);
+    const int at = rm_Q[r] + li;
+    if (at >= 0 && at < E + R - 1) p.rank_seg_idx[at] = a;
+    if (rep[u]) p.replica_seg[rpos++] = a;
+  }
+  // first segment of each expert (the first key at or above e << 21)
+  for (int e = t; e <= E; e += kThreads) {
+    int lo = 0, hi = nseg;
+    const uint32_t want = (uint32_t)e << 21;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (skeys[mid] < want) lo = mid + 1; else hi = mid;
+    }
+    p.expert_seg_ptr[e] = lo;
+  }
+  if (t == 0) {
+    *p.num_seg = nseg;
+    *p.num_replicas = nrep_tot;
+    if (p.max_rank_replicas != nullptr) *p.max_rank_replicas = mx;
+  }
+}
+
 __device__ __forceinline__ bool plan_sync(const PlanParams &p, int k) {
   if (p.nb == 1) {
     __syncthreads();
@@ -200,7 +591,7 @@ __global__ void __launch_bounds__(kThreads, 1) plan_kernel(PlanParams p) {
 
   // Tile and warp ranges (the coordinator has none).
   const int64_t b0 = coord ? 0 : (int64_t)tile * p.ppb;
-  const int64_t b1 = coord ? 0 : min(b0 + p.ppb, p.NK);
+  const int64_t b1 = coord ? 0 : min(b0 + p.ppb, p.NKt);
   const int64_t n = b1 > b0 ? b1 - b0 : 0;
   const int64_t w0 = b0 + (n * warp) / kWarps;
   const int64_t w1 = b0 + (n * (warp + 1)) / kWarps;
@@ -312,7 +703,7 @@ __global__ void __launch_bounds__(kThreads, 1) plan_kernel(PlanParams p) {
         }
       }
       const int total = __shfl_sync(0xffffffffu, incl, 31);
-      if (lane == 0) __stcg(p.counts + e, total);
+      if (lane == 0) __stcg(p.totals + e, total);
     }
   }
 
@@ -320,12 +711,31 @@ __global__ void __launch_bounds__(kThreads, 1) plan_kernel(PlanParams p) {
 
   // ---- phase 3: offsets, scalars, segments, scatter -------------------------
   // Both loads issued together: one L2 round trip before the scans.
-  const int T = t < E ? (direct ? s_T[t] : __ldcg(p.counts + t)) : 0;
-  const int tile_off =
+  const int Tt = t < E ? (direct ? s_T[t] : __ldcg(p.totals + t)) : 0;
+  int tile_off =
       (p.full && !coord && t < E)
           ? (direct ? s_pre[t] : __ldcg(p.tile + (int64_t)t * p.nt + tile))
           : 0;
-  if (direct && blockIdx.x == 0 && t < E) p.counts[t] = T;
+  int T = Tt;
+  if (p.rank_counts != nullptr) {
+    // One rank's share: T_e is the sum of the ranks' histograms, and the
+    // rank's pairs of e follow those of the ranks before it (g = r*S + s is
+    // rank-major).  The rank's own row must match what its tiles counted.
+    int sum = 0, before = 0;
+    bool mismatch = false;
+    if (t < E) {
+      for (int r = 0; r < p.R; ++r) {
+        const int v = __ldg(p.rank_counts + (int64_t)r * E + t);
+        if (r < p.rank) before += v;
+        if (r == p.rank && v != Tt) mismatch = true;
+        sum += v;
+      }
+    }
+    T = sum;
+    tile_off += before;
+    if (mismatch) set_status(p.status, MEP_ERR_DEVICE_DATA);
+  }
+  if ((direct || p.rank_counts != nullptr) && blockIdx.x == 0 && t < E) p.counts[t] = T;
   int total;
   const int off = block_excl_scan(T, &total, s_w);
   if (t < E) s_off[t] = off;
@@ -335,8 +745,8 @@ __global__ void __launch_bounds__(kThreads, 1) plan_kernel(PlanParams p) {
   if (blockIdx.x == 0) {
     const int mx = block_max(T, s_w);
     if (t == 0) {
-      *p.max_count = mx;
-      *p.maxvio = (double)((long long)mx * E) / (double)p.NK - 1.0;
+      if (p.max_count != nullptr) *p.max_count = mx;
+      if (p.maxvio != nullptr) *p.maxvio = (double)((long long)mx * E) / (double)p.NK - 1.0;
     }
   }
 
@@ -445,7 +855,7 @@ __global__ void __launch_bounds__(kThreads, 1) plan_kernel(PlanParams p) {
         }
         p.rank_seg_ptr[r] = ptr;
       }
-    } else {
+    } else if (p.kind == kPlanHomeFirst) {
       int *s_rsp = s_tab[7];
       const int R = p.R;
       // Per rank: home pieces (home experts keeping pairs) + replica pieces
@@ -519,13 +929,42 @@ __global__ void __launch_bounds__(kThreads, 1) plan_kernel(PlanParams p) {
         *p.num_seg = nseg;
         *p.num_replicas = nrep;
       }
+    } else {  // kPlanCapped: the coordinator (never a tile block) builds the tables
+      if (t < E) p.expert_offset[t] = off;
+      if (t == 0) p.expert_offset[E] = total;
+      capped_build(p, T, s_off, smem, s_w);
+    }
+  }
+
+  // The capped plan's tables reach the tile blocks through the workspace,
+  // after one more grid barrier: per expert h_e, its home slot base and its
+  // first piece; per piece its first overflow index and slot base.
+  const bool cap = p.full && p.kind == kPlanCapped;
+  int *s_ch = s_tab[1], *s_chb = s_tab[2], *s_cpb = s_tab[3];
+  int *s_cpq = &s_tab[4][0], *s_cpbase = &s_tab[4][0] + 2 * kTab;
+  if (cap) {
+    if (!plan_sync(p, direct ? 2 : 3)) return;
+    if (!coord) {
+      const int *tab_h = p.tab, *tab_hb = tab_h + E, *tab_pb = tab_hb + E;
+      const int *tab_pq = tab_pb + E + 1, *tab_pbase = tab_pq + (E + p.R);
+      const int npieces = min(__ldcg(tab_pb + E), 2 * kTab);
+      for (int i = t; i < E; i += kThreads) {
+        s_ch[i] = __ldcg(tab_h + i);
+        s_chb[i] = __ldcg(tab_hb + i);
+        s_cpb[i] = __ldcg(tab_pb + i);
+      }
+      if (t == 0) s_cpb[E] = npieces;
+      for (int i = t; i < npieces; i += kThreads) {
+        s_cpq[i] = __ldcg(tab_pq + i);
+        s_cpbase[i] = __ldcg(tab_pbase + i);
+      }
     }
   }
 
   if (p.full && !coord) {
     // Per expert: where this tile's pairs start in the expert-sorted order
     // (expert offset + tile offset); wh keeps the warp offsets in the tile.
-    int *s_base = s_tab[7];
+    int *s_base = cap ? s_rank : s_tab[7];
     __syncthreads();  // a single block has finished the coordinator's tables
     if (t < E) s_base[t] = off + tile_off;
     __syncthreads();
@@ -533,8 +972,8 @@ __global__ void __launch_bounds__(kThreads, 1) plan_kernel(PlanParams p) {
     const bool hf = p.kind == kPlanHomeFirst;
     const unsigned lt = lanemask_lt();
     const unsigned nk = (unsigned)p.NK;
-    int32_t *slot_w = p.slot + w0;
-    const int q0 = (int)w0;
+    int32_t *slot_w = p.slot + p.pair0 + w0;
+    const int q0 = (int)(p.pair0 + w0);  // global pair index of the warp's first pair
     for (int c = 0; c < nw; c += 32) {
       const int i = c + lane;
       const bool act = i < nw;
@@ -548,6 +987,7 @@ __global__ void __launch_bounds__(kThreads, 1) plan_kernel(PlanParams p) {
         const int r = wo + __popc(peers & lt);  // rank among the tile's pairs of e
         int s = s_base[e] + r;                  // position in the expert-sorted order
         if (hf) s = home_first_slot(e, s - s_off[e], Bx, C, p.R, s_h, s_off, s_O, s_F, s_D, s_rf);
+        if (cap) s = capped_slot(e, s - s_off[e], s_ch, s_chb, s_cpb, s_cpq, s_cpbase);
         slot_w[i] = s;
         if ((unsigned)s < nk) p.src_pair[s] = q0 + i;
         if (lane == __ffs(peers) - 1) wh[e] = wo + __popc(peers);
@@ -596,7 +1036,11 @@ size_t plan_workspace_bytes(const mep_shape_t &s) {
 }
 
 cudaError_t launch_plan(const mep_shape_t &s, const int32_t *idx, const mep_plan_t &pl,
-                        int full, int kind, void *ws, uint64_t wait_ns, cudaStream_t stream) {
+                        int full, int kind, void *ws, uint64_t wait_ns, cudaStream_t stream,
+                        const PlanExtra *extra) {
+  const PlanExtra none{};
+  const PlanExtra &x = extra != nullptr ? *extra : none;
+  const bool ranked = x.rank_counts != nullptr;
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
@@ -608,11 +1052,22 @@ cudaError_t launch_plan(const mep_shape_t &s, const int32_t *idx, const mep_plan
     return err;
   const int max_blocks = d.max_blocks.load(std::memory_order_relaxed);
   const int64_t NK = (int64_t)s.R * s.S * s.K;
-  int64_t want = (NK + kPlanMinPairsPerBlock - 1) / kPlanMinPairsPerBlock;
-  // One block for a single tile; otherwise a coordinator plus nt tiles.
-  const int64_t cap = std::min(max_blocks, kPlanMaxBlocks) - 1;
+  const int64_t NKt = ranked ? (int64_t)s.S * s.K : NK;  // pairs the tiles cover
+  int64_t want = (NKt + kPlanMinPairsPerBlock - 1) / kPlanMinPairsPerBlock;
+  // One block for a single tile; otherwise a coordinator plus nt tiles.  The
+  // capped plan always has a coordinator (it builds the tables in its free
+  // shared memory), and keeps the last kPlanCappedTabRows tile-matrix rows'
+  // worth of workspace for the tables it publishes.
+  const bool capped = full && kind == kPlanCapped;
+  int64_t cap = std::min(max_blocks, kPlanMaxBlocks) - 1;
+  if (ranked) cap = std::min<int64_t>(cap, kPlanTotalsRow);
+  if (capped) {
+    cap = std::min<int64_t>(cap, kPlanMaxBlocks - kPlanCappedTabRows);
+    if (cap < 1) return cudaErrorInvalidConfiguration;
+    if (capped_tab_words(s.E, s.R) > (int64_t)s.E * kPlanCappedTabRows) return cudaErrorInvalidValue;
+  }
   const int nt = (int)std::max<int64_t>(1, std::min<int64_t>(want, cap));
-  const int nb = nt > 1 ? nt + 1 : 1;
+  const int nb = (nt > 1 || capped) ? nt + 1 : 1;
   PlanParams p{};
   p.idx = idx;
   p.R = s.R; p.S = s.S; p.E = s.E; p.K = s.K;
@@ -620,7 +1075,11 @@ cudaError_t launch_plan(const mep_shape_t &s, const int32_t *idx, const mep_plan
   p.SK = (int64_t)s.S * s.K;
   p.nb = nb;
   p.nt = nt;
-  p.ppb = (NK + nt - 1) / nt;
+  p.ppb = (NKt + nt - 1) / nt;
+  p.NKt = NKt;
+  p.pair0 = ranked ? (int64_t)x.rank * s.S * s.K : 0;
+  p.rank_counts = x.rank_counts;
+  p.rank = x.rank;
   p.full = full;
   p.kind = kind;
   p.rank_seg_idx = pl.rank_seg_idx;
@@ -632,6 +1091,10 @@ cudaError_t launch_plan(const mep_shape_t &s, const int32_t *idx, const mep_plan
   p.bar = reinterpret_cast<uint32_t *>(ws);
   p.tile = reinterpret_cast<int32_t *>(static_cast<char *>(ws) + kPlanWsHeader);
   p.wait_ns = wait_ns;
+  p.B = x.B;
+  p.max_rank_replicas = x.max_rank_replicas;
+  p.tab = p.tile + (int64_t)s.E * (kPlanMaxBlocks - kPlanCappedTabRows);
+  p.totals = ranked ? p.tile + (int64_t)s.E * kPlanTotalsRow : pl.counts;
 
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(nb);

@@ -1,6 +1,11 @@
 // Backward reduction of replica weight-gradients into their home expert:
-//   home[e, :] = sum over expert e's segments s (ascending) of G[s, :]
-// in float32, zero for an expert with no segment.
+//   home[e, :] = float32( sum over expert e's segments s (ascending) of G[s, :] )
+// with the sum taken in binary64 and rounded once to float32 (nearest-even);
+// zero for an expert with no segment.  Every float32 is exact in binary64, so
+// the result is the correctly rounded value of the ascending binary64 sum,
+// whatever the cancellation between rows (a float32 running sum can be far
+// off its relative bound there).  The kernel stays bound by HBM bandwidth:
+// one conversion and one FP64 add per float read.
 //
 // Method: during the backward pass the gradients of an expert's duplicates are
 // summed into the copy on its home rank (MoonEP release page, "How MoonEP
@@ -12,10 +17,10 @@
 // of one row, so each thread owns kU vectors spaced kThreads apart (every
 // warp access is a contiguous 512-byte run).  Blocks stride over tasks,
 // expert-major; the segment range is read once per task.  A thread issues
-// the kU loads of kSU segment rows before adding them, in segment order.  G is read once and home written once,
-// both with streaming (evict-first) accesses.  The segment pointers are read
-// on the device and bounds-checked; nothing is sized from a host copy of the
-// plan.
+// the kU loads of kSU segment rows before adding them, in segment order.  G
+// is read once and home written once, both with streaming (evict-first)
+// accesses.  The segment pointers are read on the device and bounds-checked;
+// nothing is sized from a host copy of the plan.
 //
 // Rank-addressed form (mep_reduce_replica_grads_ranked): the gradients of a
 // rank's segments live in that rank's own buffer (on a multi-GPU system, a
@@ -79,10 +84,37 @@ __device__ __forceinline__ float4 zero_v<float4>() { return make_float4(0.f, 0.f
 template <>
 __device__ __forceinline__ float zero_v<float>() { return 0.f; }
 
-__device__ __forceinline__ float4 addv(float4 a, float4 b) {
-  return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
+// Binary64 accumulator of one vector of G.
+struct double4_t {
+  double x, y, z, w;
+};
+template <typename V>
+struct Acc;
+template <>
+struct Acc<float4> {
+  using T = double4_t;
+};
+template <>
+struct Acc<float> {
+  using T = double;
+};
+
+__device__ __forceinline__ void zero_acc(double4_t &a) { a.x = a.y = a.z = a.w = 0.0; }
+__device__ __forceinline__ void zero_acc(double &a) { a = 0.0; }
+
+__device__ __forceinline__ void add_acc(double4_t &a, const float4 &b) {
+  a.x = __dadd_rn(a.x, (double)b.x);
+  a.y = __dadd_rn(a.y, (double)b.y);
+  a.z = __dadd_rn(a.z, (double)b.z);
+  a.w = __dadd_rn(a.w, (double)b.w);
 }
-__device__ __forceinline__ float addv(float a, float b) { return a + b; }
+__device__ __forceinline__ void add_acc(double &a, float b) { a = __dadd_rn(a, (double)b); }
+
+__device__ __forceinline__ float4 round_acc(const double4_t &a) {
+  return make_float4(__double2float_rn(a.x), __double2float_rn(a.y), __double2float_rn(a.z),
+                     __double2float_rn(a.w));
+}
+__device__ __forceinline__ float round_acc(double a) { return __double2float_rn(a); }
 
 // Address of segment s's gradient row: row s of G, or (ranked form) the row
 // resolved into s_rows for this task (nullptr if it could not be resolved).
@@ -146,9 +178,9 @@ __global__ void __launch_bounds__(kThreads, MEP_REDUCE_MIN_BLOCKS) reduce_kernel
       if (!resolve_rows<V>(p, s0, s1, s_rows)) bad = true;
       __syncthreads();
     }
-    V acc[kU];
+    typename Acc<V>::T acc[kU];
 #pragma unroll
-    for (int j = 0; j < kU; ++j) acc[j] = zero_v<V>();
+    for (int j = 0; j < kU; ++j) zero_acc(acc[j]);
     int s = s0;
     for (; s + kSU <= s1; s += kSU) {
       V a[kSU][kU];
@@ -165,7 +197,7 @@ __global__ void __launch_bounds__(kThreads, MEP_REDUCE_MIN_BLOCKS) reduce_kernel
       for (int q = 0; q < kSU; ++q)
 #pragma unroll
         for (int j = 0; j < kU; ++j)
-          if (c0 + (int64_t)j * kThreads < p.cols) acc[j] = addv(acc[j], a[q][j]);
+          if (c0 + (int64_t)j * kThreads < p.cols) add_acc(acc[j], a[q][j]);
     }
     for (; s < s1; ++s) {
       const V *row = seg_row<V, kRanked>(p, G, s_rows, s, s0);
@@ -177,13 +209,13 @@ __global__ void __launch_bounds__(kThreads, MEP_REDUCE_MIN_BLOCKS) reduce_kernel
       }
 #pragma unroll
       for (int j = 0; j < kU; ++j)
-        if (c0 + (int64_t)j * kThreads < p.cols) acc[j] = addv(acc[j], a[j]);
+        if (c0 + (int64_t)j * kThreads < p.cols) add_acc(acc[j], a[j]);
     }
     V *hrow = home + (int64_t)el * p.cols;
 #pragma unroll
     for (int j = 0; j < kU; ++j) {
       const int64_t c = c0 + (int64_t)j * kThreads;
-      if (c < p.cols) __stcs(hrow + c, acc[j]);
+      if (c < p.cols) __stcs(hrow + c, round_acc(acc[j]));
     }
   }
   if (bad) set_status(p.status, MEP_ERR_DEVICE_DATA);

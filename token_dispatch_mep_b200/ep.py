@@ -11,8 +11,10 @@ top of the rank-addressed kernels of libmep:
   buffer is mapped into every other rank's address space once (CUDA IPC
   handles exchanged through the process group), and the R addresses of each
   kind go into a device pointer array;
-* the plan: one all-gather of the router ids, after which every rank computes
-  the identical plan on its own GPU;
+* the plan: each rank counts its own pairs per expert, one all-gather of those
+  R x E histograms follows, and every rank computes the identical tables and
+  its own pairs' slots on its own GPU (the ids themselves never leave their
+  rank);
 * dispatch: each rank writes its own tokens' rows straight into the owning
   ranks' receive buffers (one kernel, peer stores);
 * combine: each rank reads its tokens' K expert-output rows straight from
@@ -20,10 +22,17 @@ top of the rank-addressed kernels of libmep:
 * backward: each home rank sums its experts' segment gradients straight from
   the ranks that hold them (one kernel, peer loads).
 
-Ordering between ranks is by host barriers: a rank's stream is synchronised
-and then the process group's barrier is passed before a phase that reads or
-writes another rank's memory starts, and again before that memory is reused.
-No kernel waits on another rank's kernel.
+Ordering between ranks, before a phase that reads or writes another rank's
+memory and again before that memory is reused, takes one of two forms:
+
+* ``sync="host"`` (the default): the rank's stream is synchronised and the
+  process group's barrier is passed; no kernel waits on another rank's kernel.
+* ``sync="device"``: one mep_rank_barrier kernel on the rank's stream -- every
+  rank stores the crossing's epoch into its word of every rank's flag array
+  (mapped like the buffers) and waits, bounded by the library's wait limit,
+  for all R words of its own; the host never blocks between phases.  Its
+  kernels wait on the other ranks' kernels, so each rank must run on a GPU of
+  its own.
 """
 from __future__ import annotations
 
@@ -32,25 +41,22 @@ from dataclasses import dataclass
 import torch
 import torch.distributed as dist
 
-from . import (IpcHandle, Plan, Shape, mep_combine_ranked_tokens, mep_dispatch_ranked_tokens,
-               mep_ipc_close, mep_ipc_export, mep_ipc_open, mep_plan, mep_plan_home_first,
-               mep_read_status, mep_reduce_replica_grads_ranked, mep_status_string,
-               pointer_table)
+from . import (SCHEDULES, IpcHandle, Plan, Shape, mep_combine_ranked_tokens,
+               mep_dispatch_ranked_tokens, mep_ipc_close, mep_ipc_export, mep_ipc_open,
+               mep_plan_rank, mep_rank_barrier, mep_rank_histogram, mep_read_status,
+               mep_reduce_replica_grads_ranked, mep_status_string, pointer_table)
 
-__all__ = ["ExchangeGroup", "gather_router_ids", "local_segments", "max_local_segments"]
+__all__ = ["ExchangeGroup", "gather_counts", "gather_router_ids", "local_segments",
+           "max_local_segments"]
 
 
-def gather_router_ids(idx_local: torch.Tensor, group=None) -> torch.Tensor:
-    """All ranks' top-K expert ids ``[R*S, K]`` in global token order (rank r's
-    S rows at r*S), from each rank's own ``[S, K]`` int32 ids.  With an NCCL
-    group the gather runs on the GPU; with any other backend it goes through
-    host memory.  The result is on ``idx_local``'s device."""
+def _all_gather(t: torch.Tensor, group=None) -> torch.Tensor:
+    """Every rank's ``t`` stacked rank by rank (NCCL on the device, any other
+    backend through host memory); the result is on ``t``'s device."""
     world = dist.get_world_size(group)
-    if idx_local.dtype != torch.int32 or idx_local.dim() != 2:
-        raise TypeError("idx_local must be an int32 [S, K] tensor")
-    src = idx_local.contiguous()
+    src = t.contiguous()
     if dist.get_backend(group) == "nccl":
-        out = torch.empty((world * src.shape[0], src.shape[1]), dtype=torch.int32,
+        out = torch.empty((world * src.shape[0],) + tuple(src.shape[1:]), dtype=src.dtype,
                           device=src.device)
         dist.all_gather_into_tensor(out, src, group=group)
         return out
@@ -58,6 +64,24 @@ def gather_router_ids(idx_local: torch.Tensor, group=None) -> torch.Tensor:
     parts = [torch.empty_like(host) for _ in range(world)]
     dist.all_gather(parts, host, group=group)
     return torch.cat(parts).to(src.device)
+
+
+def gather_counts(counts_local: torch.Tensor, group=None) -> torch.Tensor:
+    """The plan's one exchange: every rank's per-expert histogram (int32
+    ``[E]``) gathered into ``[R, E]``, row r from rank r."""
+    if counts_local.dtype != torch.int32 or counts_local.dim() != 1:
+        raise TypeError("counts_local must be an int32 [E] tensor")
+    return _all_gather(counts_local.view(1, -1), group)
+
+
+def gather_router_ids(idx_local: torch.Tensor, group=None) -> torch.Tensor:
+    """All ranks' top-K expert ids ``[R*S, K]`` in global token order (rank r's
+    S rows at r*S), from each rank's own ``[S, K]`` int32 ids.  Not used by
+    the exchange (the plan needs only the histograms, ``gather_counts``); the
+    tests use it to compute the whole-range plan as a reference."""
+    if idx_local.dtype != torch.int32 or idx_local.dim() != 2:
+        raise TypeError("idx_local must be an int32 [S, K] tensor")
+    return _all_gather(idx_local, group)
 
 
 def max_local_segments(shape: Shape) -> int:
@@ -103,7 +127,7 @@ class ExchangeGroup:
     """
 
     def __init__(self, shape, H: int, P: int = 0, group=None, device=None,
-                 schedule: str = "contiguous"):
+                 schedule: str = "contiguous", B: int = 0, sync: str = "host"):
         self.shape = shape if isinstance(shape, Shape) else Shape(*shape)
         s = self.shape
         self.group = group
@@ -111,9 +135,17 @@ class ExchangeGroup:
         self.world = dist.get_world_size(group)
         if self.world != s.R:
             raise ValueError(f"group has {self.world} ranks, the shape {s.R}")
-        if schedule not in ("contiguous", "home_first"):
+        if schedule not in SCHEDULES:
             raise ValueError(f"unknown schedule {schedule!r}")
+        if schedule == "capped" and B < 1:
+            raise ValueError("the capped schedule needs B >= 1")
+        if sync not in ("host", "device"):
+            raise ValueError(f"unknown sync {sync!r}")
         self.schedule = schedule
+        self.sync = sync
+        self.epoch = 0            # device barrier crossings so far
+        self.B = int(B)
+        self.gathered_bytes = 0   # bytes the last plan exchanged (R x E int32)
         self.H, self.P = int(H), int(P)
         self.device = torch.device(device) if device is not None else \
             torch.device("cuda", torch.cuda.current_device())
@@ -128,6 +160,10 @@ class ExchangeGroup:
         self.recv_table = self._share(self.recv)
         self.y_table = self._share(self.y)
         self.grad_table = self._share(self.grads)
+        if sync == "device":
+            # word r of every rank's array: rank r's last crossing
+            self.flags = torch.zeros(s.R, dtype=torch.int32, device=self.device)
+            self.flag_table = self._share(self.flags)
 
     # ------------------------------------------------------------ mapping
     def _share(self, t: torch.Tensor) -> torch.Tensor:
@@ -148,6 +184,17 @@ class ExchangeGroup:
         return pointer_table(ptrs, self.device)
 
     def barrier(self):
+        """Every rank's work so far done before anything later on this rank's
+        stream: a host barrier, or the device barrier (sync="device"), whose
+        errors land in the plan's status word (``check``)."""
+        if self.sync == "device":
+            self.epoch += 1
+            mep_rank_barrier(self.flag_table, self.flags, self.rank, self.epoch,
+                             self.plan.status_tensor)
+            return
+        self.host_barrier()
+
+    def host_barrier(self):
         """This rank's GPU work done, then every rank at the same point."""
         if self.device.type == "cuda":
             torch.cuda.current_stream(self.device).synchronize()
@@ -164,12 +211,15 @@ class ExchangeGroup:
         return self.rank * self.shape.S
 
     def make_plan(self, idx_local: torch.Tensor) -> Plan:
-        """Gather every rank's router ids and compute the (identical) plan."""
-        idx = gather_router_ids(idx_local.to(self.device), self.group)
-        if self.schedule == "contiguous":
-            mep_plan(self.shape, idx, self.plan)
-        else:
-            mep_plan_home_first(self.shape, idx, self.plan)
+        """Count this rank's pairs per expert, gather every rank's histogram
+        and compute the plan's tables (identical on every rank) and this
+        rank's own pairs' slots."""
+        idx = idx_local.to(self.device).contiguous()
+        counts = mep_rank_histogram(self.shape, idx, plan=self.plan)
+        all_counts = gather_counts(counts, self.group)
+        self.gathered_bytes = all_counts.numel() * all_counts.element_size()
+        self.max_rank_replicas = mep_plan_rank(self.shape, self.schedule, self.rank, idx,
+                                               all_counts, self.plan, B=self.B)
         return self.plan
 
     def dispatch(self, x_local: torch.Tensor) -> torch.Tensor:
@@ -203,7 +253,7 @@ class ExchangeGroup:
 
     def close(self):
         """Unmap the peers' buffers (after every rank's last exchange)."""
-        self.barrier()
+        self.host_barrier()
         for m in self._mapped:
             mep_ipc_close(m.handle, m.ptr, self.device)
         self._mapped.clear()
