@@ -98,6 +98,22 @@ def test_reduced_every_element(ora, name, S, H, P):
 
 # --------------------------------------------------------------- full sizes
 
+def _combine_f64_bf16(y, w, slot):
+    """sum_k w[g,k] * y[slot[g,k]] for a chunk of tokens, added in binary64 in
+    k order (each product is exact, as in the oracle), then rounded once to
+    bf16: round-to-odd to float32, then nearest-even to bf16 (Boldo and
+    Melquiond: 16 extra bits make the two steps one correct rounding)."""
+    acc = torch.zeros((w.shape[0], y.shape[1]), dtype=torch.float64, device=y.device)
+    for k in range(w.shape[1]):
+        acc = acc + w[:, k:k + 1].double() * y.index_select(0, slot[:, k]).double()
+    f = acc.to(torch.float32)                                    # nearest-even
+    over = f.double().abs() > acc.abs()
+    fz = torch.where(over, torch.nextafter(f, torch.zeros_like(f)), f)   # toward zero
+    bits = fz.view(torch.int32)
+    bits = torch.where(fz.double() != acc, bits | 1, bits)              # sticky bit
+    return bits.view(torch.float32).to(torch.bfloat16)
+
+
 # Workloads whose every output element is compared at full size (the oracle
 # runs them in seconds); the others are compared on samples.
 EVERY_ELEMENT = ("tiny_r4_e16", "r8_e64_h2048")
@@ -141,6 +157,20 @@ def test_full_size(ora, name):
                 parity.check_reduce(home[:, c0:c1].cpu().numpy(), hexact, habs,
                                     np.diff(pl["expert_seg_ptr"]), f"{name} columns {c0}..{c1}")
         return
+    # every combine output against a float64 recomputation from the oracle's
+    # slots, in chunks on the device (the oracle itself checks a sample below)
+    wd = torch.from_numpy(np.asarray(w, np.float32)).to(DEV)
+    slot_d = torch.from_numpy(pl["slot"].astype(np.int64)).to(DEV)
+    yv = y.view(NK, H)
+    step_t = max(1, (1 << 28) // (K * H * 8))
+    for t0 in range(0, N, step_t):
+        t1 = min(N, t0 + step_t)
+        want = _combine_f64_bf16(yv, wd[t0:t1], slot_d[t0:t1])
+        got = out[t0:t1].view(torch.int16)
+        if not torch.equal(got, want.view(torch.int16)):
+            bad = int((got != want.view(torch.int16)).sum())
+            raise AssertionError(f"{name}: {bad} combine outputs differ from the float64 "
+                                 f"recomputation in tokens {t0}..{t1}")
     # combine on sampled tokens
     rng = np.random.default_rng(5)
     toks = np.unique(np.concatenate([np.arange(64), np.arange(N - 64, N), rng.integers(0, N, 512)]))

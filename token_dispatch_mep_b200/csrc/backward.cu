@@ -81,6 +81,7 @@ __device__ __forceinline__ void unpack8(const uint4 &v, float (&f)[8]) {
 
 template <int KC>
 __global__ void __launch_bounds__(kThreads) combine_bwd_kernel(CombineBwdParams p) {
+  griddep_wait();  // the previous kernel on the stream is complete and visible
   constexpr int KG = KC < 8 ? KC : 8;  // expert-output chunks loaded together
   const int lane = threadIdx.x & 31;
   const int64_t nwarps = (int64_t)gridDim.x * kWarps;
@@ -159,8 +160,7 @@ cudaError_t launch_kc(const CombineBwdParams &p, int sms, cudaStream_t stream) {
   const int64_t want = (p.N + kWarps - 1) / kWarps;
   const int blocks = (int)std::max<int64_t>(
       1, std::min<int64_t>(want, (int64_t)sms * MEP_COMBINE_BWD_BLOCKS_PER_SM));
-  combine_bwd_kernel<KC><<<blocks, kThreads, 0, stream>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(combine_bwd_kernel<KC>, dim3(blocks), dim3(kThreads), 0, stream, p);
 }
 
 }  // namespace

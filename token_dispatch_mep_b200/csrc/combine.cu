@@ -192,6 +192,7 @@ __device__ __forceinline__ const uint16_t *slot_row(const CombineParams &p, int6
 
 template <int KC, bool kRanked>
 __global__ void __launch_bounds__(kThreads, MEP_COMBINE_MIN_BLOCKS) combine_row_kernel(CombineParams p) {
+  griddep_wait();  // the previous kernel on the stream is complete and visible
   constexpr int KG = KC < 8 ? KC : 8;
   constexpr int kRU = MEP_COMBINE_ROW_U;
   const int lane = threadIdx.x & 31;
@@ -281,10 +282,8 @@ cudaError_t launch_kc(const CombineParams &p, int sms, cudaStream_t stream) {
   const int64_t want = (p.N + kWarps - 1) / kWarps;
   const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>(want, (int64_t)sms * 1024));
   if (p.rank_ys != nullptr)
-    combine_row_kernel<KC, true><<<blocks, kThreads, 0, stream>>>(p);
-  else
-    combine_row_kernel<KC, false><<<blocks, kThreads, 0, stream>>>(p);
-  return cudaGetLastError();
+    return launch_pdl(combine_row_kernel<KC, true>, dim3(blocks), dim3(kThreads), 0, stream, p);
+  return launch_pdl(combine_row_kernel<KC, false>, dim3(blocks), dim3(kThreads), 0, stream, p);
 }
 
 }  // namespace

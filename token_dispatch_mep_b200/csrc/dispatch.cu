@@ -76,6 +76,7 @@ struct DispatchParams {
 
 template <int KC, bool kRanked>
 __global__ void __launch_bounds__(kThreads) dispatch_kernel(DispatchParams p) {
+  griddep_wait();  // the previous kernel on the stream is complete and visible
   const int lane = threadIdx.x & 31;
   const int64_t nwarps = (int64_t)gridDim.x * kWarps;
   const int64_t ntask = p.N * p.parts;
@@ -189,10 +190,8 @@ cudaError_t launch_kc(const DispatchParams &p, const DispatchDev &d, cudaStream_
       1, std::min<int64_t>(want, (int64_t)d.sms * MEP_DISPATCH_BLOCKS_PER_SM));
   const int smem = d.smem.load(std::memory_order_relaxed);
   if (p.rank_bufs != nullptr)
-    dispatch_kernel<KC, true><<<blocks, kThreads, smem, stream>>>(p);
-  else
-    dispatch_kernel<KC, false><<<blocks, kThreads, smem, stream>>>(p);
-  return cudaGetLastError();
+    return launch_pdl(dispatch_kernel<KC, true>, dim3(blocks), dim3(kThreads), (size_t)smem, stream, p);
+  return launch_pdl(dispatch_kernel<KC, false>, dim3(blocks), dim3(kThreads), (size_t)smem, stream, p);
 }
 
 }  // namespace

@@ -19,6 +19,14 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
   return t;
 }
 
+// Programmatic dependent launch: a kernel launched with launch_pdl may start
+// (launch, block scheduling, prologue) while the previous kernel on its stream
+// drains; every such kernel calls griddep_wait() before its first global
+// memory access, which returns once the previous kernel has completed and its
+// writes are visible -- so results are exactly those of plain stream order.
+// Without the launch attribute the wait is a no-op.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // First error wins.
 __device__ __forceinline__ void set_status(int32_t *status, int code) {
   if (status != nullptr) atomicCAS(status, 0, code);

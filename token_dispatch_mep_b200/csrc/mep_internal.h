@@ -10,6 +10,24 @@
 
 namespace mep {
 
+// Launches `kernel` on `stream` with programmatic stream serialisation
+// allowed (see griddep_wait in mep_device.cuh).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 constexpr int kPlanThreads = 1024;
 constexpr int kPlanMaxBlocks = 1024;          // bound used to size the workspace
 constexpr int kPlanIdsPerWarp = 448;          // expert ids a plan warp keeps in shared memory

@@ -39,6 +39,7 @@ struct PrefetchParams {
 };
 
 __global__ void __launch_bounds__(kThreads) prefetch_kernel(PrefetchParams p) {
+  griddep_wait();  // the previous kernel on the stream is complete and visible
   int nrep = __ldg(p.num_replicas);
   bool bad = false;
   if (nrep < 0 || nrep > p.rows) {
@@ -101,8 +102,7 @@ cudaError_t launch_prefetch(const mep_shape_t &s, const mep_plan_t &pl, int64_t 
   const int64_t bound = (int64_t)p.rows * ((p.cols + tile - 1) / tile);
   const int blocks = (int)std::max<int64_t>(
       1, std::min<int64_t>(bound, (int64_t)sms * MEP_PREFETCH_BLOCKS_PER_SM));
-  prefetch_kernel<<<blocks, kThreads, 0, stream>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(prefetch_kernel, dim3(blocks), dim3(kThreads), 0, stream, p);
 }
 
 }  // namespace mep

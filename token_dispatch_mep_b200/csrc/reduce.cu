@@ -157,6 +157,7 @@ __device__ bool resolve_rows(const ReduceParams &p, int s0, int s1, const V **s_
 
 template <typename V, bool kRanked>
 __global__ void __launch_bounds__(kThreads, MEP_REDUCE_MIN_BLOCKS) reduce_kernel(ReduceParams p) {
+  griddep_wait();  // the previous kernel on the stream is complete and visible
   __shared__ const V *s_rows[kRanked ? kMaxSegPerExpert : 1];
   const V *G = reinterpret_cast<const V *>(p.G);
   V *home = reinterpret_cast<V *>(p.home);
@@ -236,10 +237,8 @@ cudaError_t launch(ReduceParams &p, int64_t P, cudaStream_t stream) {
   const int blocks =
       (int)std::max<int64_t>(1, std::min<int64_t>(ntask, (int64_t)sms * MEP_REDUCE_BLOCKS_PER_SM));
   if (vec)
-    reduce_kernel<float4, kRanked><<<blocks, kThreads, 0, stream>>>(p);
-  else
-    reduce_kernel<float, kRanked><<<blocks, kThreads, 0, stream>>>(p);
-  return cudaGetLastError();
+    return launch_pdl(reduce_kernel<float4, kRanked>, dim3(blocks), dim3(kThreads), 0, stream, p);
+  return launch_pdl(reduce_kernel<float, kRanked>, dim3(blocks), dim3(kThreads), 0, stream, p);
 }
 
 }  // namespace
