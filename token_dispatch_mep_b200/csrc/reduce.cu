@@ -47,6 +47,9 @@
 #ifndef MEP_REDUCE_SEG_UNROLL
 #define MEP_REDUCE_SEG_UNROLL 2  // segment rows in flight per thread
 #endif
+#ifndef MEP_REDUCE_IMAP
+#define MEP_REDUCE_IMAP 0  // 1: float32 -> binary64 by integer ops (x * 2^-896), one conversion per output
+#endif
 
 namespace mep {
 
@@ -102,19 +105,64 @@ struct Acc<float> {
 __device__ __forceinline__ void zero_acc(double4_t &a) { a.x = a.y = a.z = a.w = 0.0; }
 __device__ __forceinline__ void zero_acc(double &a) { a = 0.0; }
 
-__device__ __forceinline__ void add_acc(double4_t &a, const float4 &b) {
+#if MEP_REDUCE_IMAP
+// The float32 bits u placed at the top of a binary64 word (sign to bit 63,
+// exponent to the low end of the exponent field, fraction to the top of the
+// fraction) give exactly x * 2^-896 for every finite x, subnormals included.
+// Sums of such values round exactly like the unscaled sums: a partial sum
+// below 2^-1022 is a multiple of 2^-1045 (2^-896 times float32's finest
+// step), hence exact in both.  Infinities and NaNs do not survive the
+// mapping: *nf keeps the smallest inverted exponent seen (zero for an
+// all-ones exponent), and such a column is summed again exactly.
+__device__ __forceinline__ double f32_scaled_f64(float f, uint32_t *nf) {
+  const uint32_t u = __float_as_uint(f);
+  *nf = min(*nf, (~u) & 0x7f800000u);
+  return __hiloint2double((int)(((int32_t)u >> 3) & (int32_t)0x8fffffffu), (int)(u << 29));
+}
+__device__ __forceinline__ void add_acc(double4_t &a, const float4 &b, uint32_t *nf) {
+  a.x = __dadd_rn(a.x, f32_scaled_f64(b.x, nf));
+  a.y = __dadd_rn(a.y, f32_scaled_f64(b.y, nf));
+  a.z = __dadd_rn(a.z, f32_scaled_f64(b.z, nf));
+  a.w = __dadd_rn(a.w, f32_scaled_f64(b.w, nf));
+}
+__device__ __forceinline__ void add_acc(double &a, float b, uint32_t *nf) {
+  a = __dadd_rn(a, f32_scaled_f64(b, nf));
+}
+__device__ __forceinline__ float4 round_acc(const double4_t &a) {
+  return make_float4(__double2float_rn(a.x * 0x1p896), __double2float_rn(a.y * 0x1p896),
+                     __double2float_rn(a.z * 0x1p896), __double2float_rn(a.w * 0x1p896));
+}
+__device__ __forceinline__ float round_acc(double a) { return __double2float_rn(a * 0x1p896); }
+#else
+__device__ __forceinline__ void add_acc(double4_t &a, const float4 &b, uint32_t *) {
   a.x = __dadd_rn(a.x, (double)b.x);
   a.y = __dadd_rn(a.y, (double)b.y);
   a.z = __dadd_rn(a.z, (double)b.z);
   a.w = __dadd_rn(a.w, (double)b.w);
 }
-__device__ __forceinline__ void add_acc(double &a, float b) { a = __dadd_rn(a, (double)b); }
-
+__device__ __forceinline__ void add_acc(double &a, float b, uint32_t *) {
+  a = __dadd_rn(a, (double)b);
+}
 __device__ __forceinline__ float4 round_acc(const double4_t &a) {
   return make_float4(__double2float_rn(a.x), __double2float_rn(a.y), __double2float_rn(a.z),
                      __double2float_rn(a.w));
 }
 __device__ __forceinline__ float round_acc(double a) { return __double2float_rn(a); }
+#endif
+
+// Exact (conversion) forms, for a column that held an infinity or NaN.
+__device__ __forceinline__ void add_exact(double4_t &a, const float4 &b) {
+  a.x = __dadd_rn(a.x, (double)b.x);
+  a.y = __dadd_rn(a.y, (double)b.y);
+  a.z = __dadd_rn(a.z, (double)b.z);
+  a.w = __dadd_rn(a.w, (double)b.w);
+}
+__device__ __forceinline__ void add_exact(double &a, float b) { a = __dadd_rn(a, (double)b); }
+__device__ __forceinline__ float4 round_exact(const double4_t &a) {
+  return make_float4(__double2float_rn(a.x), __double2float_rn(a.y), __double2float_rn(a.z),
+                     __double2float_rn(a.w));
+}
+__device__ __forceinline__ float round_exact(double a) { return __double2float_rn(a); }
 
 // Address of segment s's gradient row: row s of G, or (ranked form) the row
 // resolved into s_rows for this task (nullptr if it could not be resolved).
@@ -182,6 +230,7 @@ __global__ void __launch_bounds__(kThreads, MEP_REDUCE_MIN_BLOCKS) reduce_kernel
     typename Acc<V>::T acc[kU];
 #pragma unroll
     for (int j = 0; j < kU; ++j) zero_acc(acc[j]);
+    uint32_t nf = 0xffffffffu;
     int s = s0;
     for (; s + kSU <= s1; s += kSU) {
       V a[kSU][kU];
@@ -198,7 +247,7 @@ __global__ void __launch_bounds__(kThreads, MEP_REDUCE_MIN_BLOCKS) reduce_kernel
       for (int q = 0; q < kSU; ++q)
 #pragma unroll
         for (int j = 0; j < kU; ++j)
-          if (c0 + (int64_t)j * kThreads < p.cols) add_acc(acc[j], a[q][j]);
+          if (c0 + (int64_t)j * kThreads < p.cols) add_acc(acc[j], a[q][j], &nf);
     }
     for (; s < s1; ++s) {
       const V *row = seg_row<V, kRanked>(p, G, s_rows, s, s0);
@@ -210,13 +259,33 @@ __global__ void __launch_bounds__(kThreads, MEP_REDUCE_MIN_BLOCKS) reduce_kernel
       }
 #pragma unroll
       for (int j = 0; j < kU; ++j)
-        if (c0 + (int64_t)j * kThreads < p.cols) add_acc(acc[j], a[j]);
+        if (c0 + (int64_t)j * kThreads < p.cols) add_acc(acc[j], a[j], &nf);
     }
     V *hrow = home + (int64_t)el * p.cols;
+    if (MEP_REDUCE_IMAP && nf == 0) {
+      // an infinity or NaN among this thread's inputs: sum its columns again
+      // with exact conversions (rare; no cross-thread work involved)
 #pragma unroll
-    for (int j = 0; j < kU; ++j) {
-      const int64_t c = c0 + (int64_t)j * kThreads;
-      if (c < p.cols) __stcs(hrow + c, round_acc(acc[j]));
+      for (int j = 0; j < kU; ++j) zero_acc(acc[j]);
+      for (int s2 = s0; s2 < s1; ++s2) {
+        const V *row = seg_row<V, kRanked>(p, G, s_rows, s2, s0);
+#pragma unroll
+        for (int j = 0; j < kU; ++j) {
+          const int64_t c = c0 + (int64_t)j * kThreads;
+          if (row != nullptr && c < p.cols) add_exact(acc[j], __ldcs(row + c));
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < kU; ++j) {
+        const int64_t c = c0 + (int64_t)j * kThreads;
+        if (c < p.cols) __stcs(hrow + c, round_exact(acc[j]));
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < kU; ++j) {
+        const int64_t c = c0 + (int64_t)j * kThreads;
+        if (c < p.cols) __stcs(hrow + c, round_acc(acc[j]));
+      }
     }
   }
   if (bad) set_status(p.status, MEP_ERR_DEVICE_DATA);
