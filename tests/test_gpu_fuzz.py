@@ -1,8 +1,8 @@
 """Randomised parity (hypothesis, derandomised): small random shapes and
 routings -- skewed, duplicate ids inside a token, everything on one expert,
 ids at the edges of [0, E) -- through the C ABI on the GPU, against the
-oracle: both plans bit-exact, dispatch bit-exact, combine and reduce within
-the contract's tolerances, and one rank's token range of the rank-addressed
+oracle: the contiguous, home-first and capped plans (B from 1 to 5) bit-exact,
+dispatch, combine and reduce bit-exact, and one rank's token range of the rank-addressed
 calls (dispatch, combine, and the home rank's share of the reduction)
 equal to the whole-range results."""
 import numpy as np
@@ -67,10 +67,20 @@ def test_random_shapes_against_the_oracle(c):
     x = torch.randn((N, H), generator=gen).to(torch.bfloat16)
     y = torch.randn((NK, H), generator=gen).to(torch.bfloat16)
     G = torch.randn((E + R - 1, P), generator=gen)
-    for home_first in (False, True):
+    Bcap = 1 + seed % 5
+    for home_first in (False, True, "capped"):
         plan = mep.Plan(s, DEV)
-        (mep.mep_plan_home_first if home_first else mep.mep_plan)(s, torch.from_numpy(idx).to(DEV), plan)
-        pl = (ora.plan_home_first if home_first else ora.plan)(R, S, E, K, idx)
+        idx_d = torch.from_numpy(idx).to(DEV)
+        if home_first == "capped":
+            mr = mep.mep_plan_capped(s, Bcap, idx_d, plan)
+            pl = ora.plan_capped(R, S, E, K, Bcap, idx)
+            assert int(mr.item()) == pl["max_rank_replicas"]
+        elif home_first:
+            mep.mep_plan_home_first(s, idx_d, plan)
+            pl = ora.plan_home_first(R, S, E, K, idx)
+        else:
+            mep.mep_plan(s, idx_d, plan)
+            pl = ora.plan(R, S, E, K, idx)
         buf = torch.empty((NK, H), dtype=torch.bfloat16, device=DEV)
         out = torch.empty((N, H), dtype=torch.bfloat16, device=DEV)
         home = torch.empty((E, P), dtype=torch.float32, device=DEV)
@@ -90,7 +100,7 @@ def test_random_shapes_against_the_oracle(c):
                                       torch.from_numpy(w[r * S:(r + 1) * S].copy()).to(DEV), out_r)
         assert mep.mep_read_status(plan) == 0
         parity.check_plan(plan.host(), pl, f"fuzz hf={home_first}")
-        if not home_first:  # the counts-and-maxvio-only call on the same ids
+        if home_first is False:  # the counts-and-maxvio-only call on the same ids
             ws = torch.zeros(mep.mep_plan_workspace_bytes(s), dtype=torch.uint8, device=DEV)
             cnt = torch.empty(E, dtype=torch.int32, device=DEV)
             mc = torch.empty(1, dtype=torch.int32, device=DEV)

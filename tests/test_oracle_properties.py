@@ -1,7 +1,8 @@
 """Property-based pins of the oracle (hypothesis): on random small shapes and
 routings -- skewed, duplicated ids inside a token, all ids on one expert --
 the oracle's contiguous plan equals Python's sorted() over (expert, g, k),
-its home-first plan equals the queue simulation of the schedule, both keep
+its home-first and capped plans equal the queue simulations of their
+schedules, all keep
 the invariants that fix them (every rank exactly S*K slots, each pair placed
 once, runs of one expert, segment bound), and combine / reduce equal exact
 rational sums.  CPU only; a bounded number of examples keeps it to seconds."""
@@ -64,6 +65,15 @@ def test_home_first_plan_is_the_queue_simulation(case):
     # (Fewer replicas than the contiguous cut is typical, not a theorem: with
     # R=4, S=4, E=12, K=1 a routing exists where home-first makes 2 and the
     # contiguous cut 1, so no such bound is asserted here.)
+
+
+@SETTINGS
+@given(routed(), st.integers(1, 8))
+def test_capped_plan_is_the_queue_simulation(case, B):
+    R, S, E, K, idx = case
+    pl = ORA.plan_capped(R, S, E, K, B, idx)
+    pins._check_capped_equal(pl, pins.brute_capped(R, S, E, K, B, idx), str((R, S, E, K, B)))
+    pins.check_capped_invariants(pl, R, S, E, K, B, idx)
 
 
 @SETTINGS
