@@ -70,6 +70,9 @@ def parse_args():
                     help="skip the CUDA-graph replay timing of the step")
     ap.add_argument("--no-backward", action="store_true",
                     help="skip the separately timed backward kernels")
+    ap.add_argument("--dispatch-form", choices=["register", "bulk"], default="register",
+                    help="dispatch through registers (mep_dispatch) or the bulk-copy engine "
+                         "(mep_dispatch_bulk, the staged form kept for comparison)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle baseline sample")
     return ap.parse_args()
@@ -359,13 +362,15 @@ def main():
         flush.zero_()
         clean.sum()
 
+    dispatch = mep.mep_dispatch_bulk if args.dispatch_form == "bulk" else mep.mep_dispatch
+
     def step(evs=None):
         if evs:
             evs[0].record()
         mep.mep_plan(s, idx, plan)
         if evs:
             evs[1].record()
-        mep.mep_dispatch(s, H, plan, x, buf)
+        dispatch(s, H, plan, x, buf)
         if evs:
             evs[2].record()
         mep.mep_combine(s, H, plan, y, w, out)
@@ -637,7 +642,8 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
-            "config": bench_config(wl, world),
+            "config": dict(bench_config(wl, world), **(
+                {"dispatch_form": "bulk copy (mep_dispatch_bulk)"} if args.dispatch_form == "bulk" else {})),
             "timing": ("CUDA-graph replay of the captured step, events around each replay"
                        if graph is not None else "eager launches, events around each kernel"),
             "roofline": roofline,

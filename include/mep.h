@@ -259,6 +259,18 @@ MEP_API mep_status_t mep_plan_rank(mep_shape_t shape, int32_t schedule, int32_t 
 MEP_API mep_status_t mep_dispatch(mep_shape_t shape, int32_t H, const mep_plan_t *plan,
                           const uint16_t *x, uint16_t *buf, void *stream);
 
+/* mep_dispatch through the bulk-copy (TMA) engine: the same arguments and the
+ * same bytes in buf, with every row staged in shared memory -- one bulk load
+ * of the token's row, then K bulk stores of it to the token's slots, per
+ * pipeline of two shared-memory stages.  Kept for comparison with
+ * mep_dispatch, which moves the rows through registers and is faster on B200
+ * (0.96-0.99 of the HBM copy bandwidth against 0.83-0.86 for this form on
+ * the R=8/E=64, Kimi-shaped and R=32 skew workloads).  Its waits on row
+ * arrival are bounded by mep_get_wait_limit_ns (MEP_ERR_TIMEOUT in
+ * plan->status); a slot outside [0, N*K) records MEP_ERR_DEVICE_DATA. */
+MEP_API mep_status_t mep_dispatch_bulk(mep_shape_t shape, int32_t H, const mep_plan_t *plan,
+                                       const uint16_t *x, uint16_t *buf, void *stream);
+
 /* Weighted combine back to token order (the return leg of the top-K routing
  * in "Why expert parallelism is needed").
  *   y      bf16 [R, S*K, H] expert outputs in slot order, 16-byte aligned.

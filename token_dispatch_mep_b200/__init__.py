@@ -20,6 +20,7 @@ __all__ = [
     "MepError", "Shape", "Plan", "load_library", "library_path",
     "mep_plan_workspace_bytes", "mep_maxvio", "mep_plan", "mep_plan_home_first", "mep_plan_noalloc",
     "mep_plan_capped", "mep_rank_histogram", "mep_plan_rank", "SCHEDULES", "mep_rank_barrier",
+    "mep_dispatch_bulk",
     "mep_dispatch",
     "mep_combine", "mep_combine_backward", "mep_dispatch_backward", "mep_prefetch_replica_weights",
     "mep_dispatch_ranked", "mep_combine_ranked", "rank_pointer_table", "pointer_table",
@@ -44,7 +45,7 @@ ABI_SYMBOLS = ("mep_plan_workspace_bytes", "mep_maxvio", "mep_plan", "mep_dispat
                "mep_combine_ranked", "mep_dispatch_ranked_tokens", "mep_combine_ranked_tokens",
                "mep_reduce_replica_grads_ranked", "mep_ipc_export", "mep_ipc_open",
                "mep_ipc_close", "mep_plan_capped", "mep_rank_histogram", "mep_plan_rank",
-               "mep_rank_barrier")
+               "mep_rank_barrier", "mep_dispatch_bulk")
 
 
 class MepError(RuntimeError):
@@ -116,6 +117,7 @@ def load_library():
         "mep_maxvio": ([Shape, vp, vp, vp, vp, vp, vp, sz, vp], ctypes.c_int),
         "mep_plan": ([Shape, vp, P, vp, sz, vp], ctypes.c_int),
         "mep_dispatch": ([Shape, i32, P, vp, vp, vp], ctypes.c_int),
+        "mep_dispatch_bulk": ([Shape, i32, P, vp, vp, vp], ctypes.c_int),
         "mep_combine": ([Shape, i32, P, vp, vp, vp, vp], ctypes.c_int),
         "mep_reduce_replica_grads": ([Shape, P, i64, vp, vp, vp], ctypes.c_int),
         "mep_read_status": ([P, vp], ctypes.c_int),
@@ -376,6 +378,17 @@ def mep_dispatch(shape, H: int, plan: Plan, x, buf):
     xp = _need(x, "x", torch.bfloat16, s.N * H, dev)
     bp = _need(buf, "buf", torch.bfloat16, s.NK * H, dev)
     _ok(L.mep_dispatch(s, int(H), ctypes.byref(plan.struct), xp, bp, _stream(dev)), "mep_dispatch")
+
+
+def mep_dispatch_bulk(shape, H: int, plan: Plan, x, buf):
+    """``mep_dispatch`` through the bulk-copy engine (rows staged in shared
+    memory); the same result, kept for comparison (slower on B200)."""
+    L, s = load_library(), _shape(shape)
+    dev = plan.device
+    xp = _need(x, "x", torch.bfloat16, s.N * H, dev)
+    bp = _need(buf, "buf", torch.bfloat16, s.NK * H, dev)
+    _ok(L.mep_dispatch_bulk(s, int(H), ctypes.byref(plan.struct), xp, bp, _stream(dev)),
+        "mep_dispatch_bulk")
 
 
 def mep_combine(shape, H: int, plan: Plan, y, topk_w, out):

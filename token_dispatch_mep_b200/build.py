@@ -14,7 +14,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libmep.so")
 OBJDIR = os.path.join(ROOT, "_build")
 SOURCES = ["abi.cu", "plan.cu", "dispatch.cu", "combine.cu", "reduce.cu", "backward.cu", "prefetch.cu",
-           "noalloc.cu", "ipc.cu", "barrier.cu"]
+           "noalloc.cu", "ipc.cu", "barrier.cu", "dispatch_bulk.cu"]
 HEADERS = ["mep_device.cuh", "mep_internal.h"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

@@ -192,6 +192,17 @@ mep_status_t mep_dispatch(mep_shape_t shape, int32_t H, const mep_plan_t *plan, 
                                         nullptr, as_stream(stream)));
 }
 
+mep_status_t mep_dispatch_bulk(mep_shape_t shape, int32_t H, const mep_plan_t *plan,
+                               const uint16_t *x, uint16_t *buf, void *stream) {
+  mep_status_t st = check_shape(shape);
+  if (st != MEP_OK) return st;
+  if ((st = check_hidden(H)) != MEP_OK) return st;
+  if (!plan || !plan->slot || !plan->status || !x || !buf) return MEP_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(buf, 16) || !aligned(plan->slot, 4)) return MEP_ERR_MISALIGNED;
+  return from_cuda(mep::launch_dispatch_bulk(shape, H, *plan, x, buf, g_wait_ns.load(),
+                                             as_stream(stream)));
+}
+
 mep_status_t mep_combine(mep_shape_t shape, int32_t H, const mep_plan_t *plan, const uint16_t *y,
                          const float *topk_w, uint16_t *out, void *stream) {
   mep_status_t st = check_shape(shape);

@@ -23,9 +23,13 @@
 //   subnormals included: the two formats' subnormal scales differ by the same
 //   2^-896), and the weight is scaled by 2^896 once per term (exact: a float32
 //   times 2^896 stays below 2^1024).  Infinities and NaNs do not survive this
-//   mapping, so every loaded word is checked for an all-ones exponent; a chunk
-//   that holds one is summed again with exact conversions (the oracle's
-//   arithmetic: inf and NaN propagate).
+//   mapping, so every loaded word's exponent fields are folded into a running
+//   16x2 maximum (one instruction per two elements; an all-ones exponent is
+//   the largest); a chunk that held one is summed again with exact
+//   conversions (the oracle's arithmetic: inf and NaN propagate).  Measured
+//   against the alternatives (float32 -> binary64 conversion instructions;
+//   one chunk per lane with more resident warps), this form moved the most
+//   bytes on every workload.
 //
 // One warp per token walks the row, kRU = 2 16-byte chunks (8 bf16 each) per
 // lane per step.  Lanes k < K hold the token's slot id and weight, which the
@@ -61,8 +65,11 @@
 #ifndef MEP_COMBINE_ROW_U
 #define MEP_COMBINE_ROW_U 2  // 16-byte chunks per lane per step
 #endif
+#ifndef MEP_COMBINE_GROUP
+#define MEP_COMBINE_GROUP 8  // expert-output loads issued together (k values per group)
+#endif
 #ifndef MEP_COMBINE_NF_MAX
-#define MEP_COMBINE_NF_MAX 0  // 1: non-finite check by a 16x2 max of the exponents
+#define MEP_COMBINE_NF_MAX 1  // 1: non-finite check by a 16x2 max of the exponents
 #endif
 #ifndef MEP_COMBINE_CVT
 #define MEP_COMBINE_CVT 0  // 1: bf16 -> float32 -> binary64 by conversion instructions
@@ -100,6 +107,7 @@ __device__ __forceinline__ double bf16_hi_to_scaled_f64(uint32_t x) {
   return __hiloint2double((int)(((int32_t)x >> 3) & (int32_t)0x8fffe000u), 0);
 }
 
+#if !MEP_COMBINE_NF_MAX
 // Nonzero in bit 15 or 31 if a bf16 half of u has an all-ones exponent
 // (infinity or NaN): the masked, inverted exponent of such a half is zero, and
 // subtracting 1 from it sets the half's top bit (no other half value, all
@@ -107,6 +115,7 @@ __device__ __forceinline__ double bf16_hi_to_scaled_f64(uint32_t x) {
 __device__ __forceinline__ uint32_t nonfinite_bits(uint32_t u) {
   return ((~u) & 0x7f807f80u) - 0x00010001u;
 }
+#endif
 
 #if MEP_COMBINE_NF_MAX
 __device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
@@ -193,7 +202,7 @@ __device__ __forceinline__ const uint16_t *slot_row(const CombineParams &p, int6
 template <int KC, bool kRanked>
 __global__ void __launch_bounds__(kThreads, MEP_COMBINE_MIN_BLOCKS) combine_row_kernel(CombineParams p) {
   griddep_wait();  // the previous kernel on the stream is complete and visible
-  constexpr int KG = KC < 8 ? KC : 8;
+  constexpr int KG = KC < MEP_COMBINE_GROUP ? KC : MEP_COMBINE_GROUP;
   constexpr int kRU = MEP_COMBINE_ROW_U;
   const int lane = threadIdx.x & 31;
   const int64_t nwarps = (int64_t)gridDim.x * kWarps;

@@ -80,6 +80,12 @@ cudaError_t launch_dispatch(const mep_shape_t &s, int32_t H, const mep_plan_t &p
                             int64_t count, const uint16_t *x, uint16_t *buf,
                             uint16_t *const *rank_bufs, cudaStream_t stream);
 
+// The bulk-copy (TMA engine) form of dispatch, same results as launch_dispatch
+// over all tokens; waits bounded by wait_ns.
+cudaError_t launch_dispatch_bulk(const mep_shape_t &s, int32_t H, const mep_plan_t &pl,
+                                 const uint16_t *x, uint16_t *buf, uint64_t wait_ns,
+                                 cudaStream_t stream);
+
 cudaError_t launch_combine(const mep_shape_t &s, int32_t H, const mep_plan_t &pl, int64_t g0,
                            int64_t count, const uint16_t *y, const uint16_t *const *rank_ys,
                            const float *w, uint16_t *out, cudaStream_t stream);

@@ -65,9 +65,6 @@ constexpr int kDirectLoads = 8;  // tile-matrix entries per thread in the direct
 #ifndef MEP_PLAN_PEERS_BALLOT
 #define MEP_PLAN_PEERS_BALLOT 1  // 1: peer masks from bit ballots; 0: match.any
 #endif
-#ifndef MEP_PLAN_FUSED_BASE
-#define MEP_PLAN_FUSED_BASE 1    // 1: expert bases folded into the warp cursors
-#endif
 
 struct PlanParams {
   const int32_t *idx;
@@ -973,15 +970,6 @@ __global__ void __launch_bounds__(kThreads, 1) plan_kernel(PlanParams p) {
     __syncthreads();
 
     const bool hf = p.kind == kPlanHomeFirst;
-#if MEP_PLAN_FUSED_BASE
-    // Fold each expert's base into the warp's own cursor row once: the
-    // position in the expert-sorted order (contiguous plan) or the index
-    // among the expert's pairs (home-first and capped plans), so the loop
-    // below reads one shared word per pair instead of two or three.
-    for (int e2 = lane; e2 < E; e2 += 32)
-      wh[e2] += (hf || cap) ? s_base[e2] - s_off[e2] : s_base[e2];
-    __syncwarp();
-#endif
     const unsigned lt = lanemask_lt();
     const unsigned nk = (unsigned)p.NK;
     int32_t *slot_w = p.slot + p.pair0 + w0;
@@ -996,19 +984,10 @@ __global__ void __launch_bounds__(kThreads, 1) plan_kernel(PlanParams p) {
       const int wo = valid ? wh[e] : 0;
       __syncwarp();
       if (valid) {
-#if MEP_PLAN_FUSED_BASE
-        // wo already holds the expert's base: the position (contiguous) or
-        // the index among the expert's pairs (home-first, capped)
-        const int r = wo + __popc(peers & lt);
-        int s = r;
-        if (hf) s = home_first_slot(e, r, Bx, C, p.R, s_h, s_off, s_O, s_F, s_D, s_rf);
-        if (cap) s = capped_slot(e, r, s_ch, s_chb, s_cpb, s_cpq, s_cpbase);
-#else
         const int r = wo + __popc(peers & lt);  // rank among the tile's pairs of e
         int s = s_base[e] + r;                  // position in the expert-sorted order
         if (hf) s = home_first_slot(e, s - s_off[e], Bx, C, p.R, s_h, s_off, s_O, s_F, s_D, s_rf);
         if (cap) s = capped_slot(e, s - s_off[e], s_ch, s_chb, s_cpb, s_cpq, s_cpbase);
-#endif
         slot_w[i] = s;
         if ((unsigned)s < nk) p.src_pair[s] = q0 + i;
         if (lane == __ffs(peers) - 1) wh[e] = wo + __popc(peers);
