@@ -48,6 +48,12 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
   return m;
 }
 
+__device__ __forceinline__ uint32_t lanemask_gt() {
+  uint32_t m;
+  asm("mov.u32 %0, %%lanemask_gt;" : "=r"(m));
+  return m;
+}
+
 __device__ __forceinline__ void red_release_add_gpu(uint32_t *p, uint32_t v) {
   asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }

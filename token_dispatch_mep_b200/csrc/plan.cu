@@ -63,7 +63,8 @@ constexpr int kTab = MEP_MAX_EXPERTS + 1;
 constexpr int kDirectLoads = 8;  // tile-matrix entries per thread in the direct phase 2
 
 #ifndef MEP_PLAN_PEERS_BALLOT
-#define MEP_PLAN_PEERS_BALLOT 1  // 1: peer masks from bit ballots; 0: match.any
+#define MEP_PLAN_PEERS_BALLOT 2  // 2: peer masks from ballots on all 11 id bits, unrolled;
+                                 // 1: the same over the id's nbits, in a loop; 0: match.any
 #endif
 
 struct PlanParams {
@@ -97,9 +98,21 @@ struct PlanParams {
   int32_t *tab;                // workspace: the scatter tables the coordinator publishes
 };
 
-// Mask of the lanes whose key equals this lane's key; keys are < 2^nbits.
+// Mask of the lanes whose key equals this lane's key; keys are < 2^nbits
+// (nbits <= 11, E <= 1024).
 __device__ __forceinline__ unsigned peers_of(int key, int nbits) {
-#if MEP_PLAN_PEERS_BALLOT
+#if MEP_PLAN_PEERS_BALLOT == 2
+  // bits at and above nbits are zero in every key: their ballots change nothing
+  (void)nbits;
+  unsigned m = 0xffffffffu;
+#pragma unroll
+  for (int b = 0; b < 11; ++b) {
+    const unsigned bit = (unsigned)(key >> b) & 1u;
+    const unsigned on = __ballot_sync(0xffffffffu, bit);
+    m &= ~(on ^ (0u - bit));  // lanes whose bit b equals this lane's
+  }
+  return m;
+#elif MEP_PLAN_PEERS_BALLOT
   unsigned m = 0xffffffffu;
   for (int b = 0; b < nbits; ++b) {
     const bool bit = (key >> b) & 1;
@@ -137,6 +150,35 @@ __device__ __forceinline__ int block_excl_scan(int v, int *total, int *s_w) {
   __syncthreads();
   const int before = warp ? s_w[warp - 1] : 0;
   *total = s_w[kWarps - 1];
+  __syncthreads();
+  return before + x - v;
+}
+
+// block_excl_scan for 64-bit values (two int-sized sums packed in one), with
+// its own shared words.
+__device__ __forceinline__ long long block_excl_scan64(long long v, long long *total) {
+  __shared__ long long s_w64[kWarps];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  long long x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const long long y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) s_w64[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    long long w = s_w64[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    s_w64[lane] = w;
+  }
+  __syncthreads();
+  const long long before = warp ? s_w64[warp - 1] : 0;
+  *total = s_w64[kWarps - 1];
   __syncthreads();
   return before + x - v;
 }
@@ -196,22 +238,51 @@ __device__ __forceinline__ int capped_slot(int e, int i, const int *s_h, const i
   return s_pbase[lo] + q;
 }
 
-// Ascending bitonic sort of n keys in shared memory (n a power of two,
-// n <= 2 * blockDim.x); every thread of the block must call it.
-template <typename K>
-__device__ void block_bitonic_sort(K *a, int n) {
-  for (int k = 2; k <= n; k <<= 1) {
+// One compare-exchange of a bitonic network, seen from position i: the key
+// it keeps against its partner's key y at distance j in merge size k.
+template <typename Key>
+__device__ __forceinline__ Key bitonic_keep(Key x, Key y, int i, int j, int k) {
+  const bool keep_min = ((i & k) == 0) == ((i & j) == 0);
+  const bool lt = x < y;
+  return keep_min == lt ? x : y;
+}
+
+// Ascending bitonic sort of n2 keys (n2 a power of two, n2 <= V * blockDim.x)
+// held in registers: thread t holds positions t and t + blockDim.x.  Steps
+// with a partner inside the warp exchange by shuffle; longer ones go through
+// shared memory (buf: 2 * n2 keys, double-buffered, one barrier per step);
+// with V = 2 the longest step pairs a thread's own two keys.  Every thread of
+// the block calls it; positions >= n2 are ignored.
+template <typename Key, int V>
+__device__ void block_sort_regs(Key (&x)[V], int n2, Key *buf) {
+  const int t = threadIdx.x;
+  int cur = 0;
+  for (int k = 2; k <= n2; k <<= 1) {
     for (int j = k >> 1; j > 0; j >>= 1) {
-      for (int i = threadIdx.x; i < (n >> 1); i += blockDim.x) {
-        const int lo = ((i & ~(j - 1)) << 1) | (i & (j - 1));
-        const int hi = lo + j;
-        const K x = a[lo], y = a[hi];
-        if ((x > y) == ((lo & k) == 0)) {
-          a[lo] = y;
-          a[hi] = x;
+      Key y[V];
+      if (j >= kThreads) {  // only with V == 2: positions t and t + kThreads
+        y[0] = x[V - 1];
+        y[V - 1] = x[0];
+      } else if (j >= 32) {
+        Key *b = buf + cur * n2;
+#pragma unroll
+        for (int u = 0; u < V; ++u) {
+          const int i = t + u * kThreads;
+          if (i < n2) b[i] = x[u];
         }
+        __syncthreads();
+#pragma unroll
+        for (int u = 0; u < V; ++u) {
+          const int i = t + u * kThreads;
+          y[u] = i < n2 ? b[i ^ j] : x[u];
+        }
+        cur ^= 1;
+      } else {
+#pragma unroll
+        for (int u = 0; u < V; ++u) y[u] = __shfl_xor_sync(0xffffffffu, x[u], j);
       }
-      __syncthreads();
+#pragma unroll
+      for (int u = 0; u < V; ++u) x[u] = bitonic_keep(x[u], y[u], t + u * kThreads, j, k);
     }
   }
 }
@@ -229,332 +300,396 @@ __host__ __device__ __forceinline__ int64_t capped_tab_words(int E, int R) {
   return 3 * (int64_t)E + 1 + 2 * ((int64_t)E + R);
 }
 
-// The capped schedule's tables, built by the coordinator block (which owns no
-// pairs, so its dynamic shared memory is free scratch: sm holds at least
-// kWarps * E + kWarps * kPlanIdsPerWarp ints, more than the 18 E + 15 R + 2 n2
-// + 8 (n2 <= 2 (E + R)) this needs, since R <= E <= 1024).  T is this thread's expert count (t < E), s_off
-// the expert offsets.  Writes every plan field except counts, offsets, slot
-// and src_pair, and publishes the scatter tables to p.tab.
-//   1. home fill, smallest home experts first (ties: lower id);
+// Shared-memory ints the capped builder uses: 13 E + 9 R + 6 (E + R) + 8,
+// plus two sort buffers of n2 8-byte keys (n2 the power of two at or above
+// the items and rooms, at most E + R).  The coordinator's dynamic shared
+// memory holds kWarps * (E + kPlanIdsPerWarp) ints, which is more for every
+// E <= MEP_MAX_EXPERTS (R <= E); the launch checks it.
+__host__ __device__ __forceinline__ int64_t capped_smem_ints(int E, int R) {
+  int64_t n2 = 1;  // sort size bound: the power of two at or above E + R
+  while (n2 < (int64_t)E + R) n2 <<= 1;
+  return 13 * (int64_t)E + 9 * (int64_t)R + 6 * ((int64_t)E + R) + 8 + 4 * n2;
+}
+
+// The capped builder's arrays in the coordinator's shared memory.
+struct CapMem {
+  int *sT;        // [E] T_e
+  int *sh;        // [E] h_e, pairs kept home
+  int *shb;       // [E] home slot base of e
+  int *shf;       // [E] home pieces of the experts before e
+  int *spb;       // [E+1] first replica piece of e
+  int *shl;       // [E] index of e's home piece among its rank's segments
+  int *it_e;      // [E] expert of item i (items: overflow descending, expert ascending)
+  int *it_O;      // [E] overflow of item i
+  int *it_loc;    // [E] filler: start in its room's replica area, else -1
+  int *it_P;      // [E] stream position of item i
+  int *it_s;      // [E] stream index, or a filler's index in its room
+  int *it_of;     // [E] item index of expert e, -1 if e has no overflow
+  int *st_i;      // [E] item at stream index s
+  int *rm_r;      // [R] rank of room j (rooms: spare room descending, rank ascending)
+  int *rm_D;      // [R] spare room
+  int *rm_left;   // [R] space left after the fillers
+  int *rm_nf;     // [R] fillers placed
+  int *rm_Q;      // [R] stream position of room j's space left; then rank_seg_ptr
+  int *rm_first;  // [R] stream index of the first item meeting room j
+  int *rm_nz;     // [R+1] rooms with space left before room j
+  int *rk_nh;     // [R] home pieces of rank r
+  int *rk_nr;     // [R] replica pieces of rank r
+  int *pc_e, *pc_r, *pc_loc, *pc_n, *pc_q, *pc_li;  // [E+R] per piece: expert, rank,
+                  // first slot within the rank, size, first overflow index, index
+                  // among the rank's segments (slot order)
+  int *misc;      // [4]: home pieces, replica pieces
+  uint64_t *keys; // [n2] sorted items and rooms (aliases the piece arrays)
+  uint64_t *sbuf; // [2 n2] sort exchange buffers
+};
+
+__device__ __forceinline__ CapMem cap_mem(int *sm, int E, int R) {
+  CapMem m;
+  const int NP = E + R;
+  int *q = sm;
+  m.sT = q; q += E;
+  m.sh = q; q += E;
+  m.shb = q; q += E;
+  m.shf = q; q += E;
+  m.spb = q; q += E + 1;
+  m.shl = q; q += E;
+  m.it_e = q; q += E;
+  m.it_O = q; q += E;
+  m.it_loc = q; q += E;
+  m.it_P = q; q += E;
+  m.it_s = q; q += E;
+  m.it_of = q; q += E;
+  m.st_i = q; q += E;
+  m.rm_r = q; q += R;
+  m.rm_D = q; q += R;
+  m.rm_left = q; q += R;
+  m.rm_nf = q; q += R;
+  m.rm_Q = q; q += R;
+  m.rm_first = q; q += R;
+  m.rm_nz = q; q += R + 1;
+  m.rk_nh = q; q += R;
+  m.rk_nr = q; q += R;
+  m.misc = q; q += 4;
+  q = reinterpret_cast<int *>((reinterpret_cast<uintptr_t>(q) + 7) & ~static_cast<uintptr_t>(7));
+  m.keys = reinterpret_cast<uint64_t *>(q);  // n2 <= 2 NP - 1 keys: inside the 6 NP piece ints
+  m.pc_e = q; q += NP;
+  m.pc_r = q; q += NP;
+  m.pc_loc = q; q += NP;
+  m.pc_n = q; q += NP;
+  m.pc_q = q; q += NP;
+  m.pc_li = q; q += NP;
+  m.sbuf = reinterpret_cast<uint64_t *>(q);  // even offset from the aligned base
+  return m;
+}
+
+// Keys of the one sort of step 2: items (overflowing experts) first by
+// overflow descending, then expert; rooms (ranks with spare room) after them
+// by room descending, then rank.
+__device__ __forceinline__ uint64_t item_key(int O, int e) {
+  return ((uint64_t)(0x7fffffff - O) << 32) | (uint32_t)e;
+}
+__device__ __forceinline__ uint64_t room_key(int D, int r) {
+  return (1ull << 63) | ((uint64_t)(0x7fffffff - D) << 32) | (uint32_t)r;
+}
+
+template <int V>
+__device__ __forceinline__ void capped_sort_and_decode(const CapMem &m, int n2, int X, int Y) {
+  const int t = threadIdx.x;
+  uint64_t x[V];
+#pragma unroll
+  for (int u = 0; u < V; ++u) {
+    const int i = t + u * kThreads;
+    x[u] = i < X + Y ? m.keys[i] : ~0ull;
+  }
+  block_sort_regs<uint64_t, V>(x, n2, m.sbuf);
+#pragma unroll
+  for (int u = 0; u < V; ++u) {
+    const int i = t + u * kThreads;
+    const int id = (int)(x[u] & 0xffffffffu);
+    const int v = 0x7fffffff - (int)((x[u] >> 32) & 0x7fffffff);
+    if (i < X) {
+      m.it_e[i] = id;
+      m.it_O[i] = v;
+      m.it_of[id] = i;
+      m.it_loc[i] = -1;
+    } else if (i < X + Y) {
+      m.rm_r[i - X] = id;
+      m.rm_D[i - X] = v;
+    }
+  }
+}
+
+// The capped schedule's scatter tables, built by the coordinator block (which
+// owns no pairs, so its dynamic shared memory is free scratch).  T is this
+// thread's expert count (t < E), s_off the expert offsets.  Writes
+// max_rank_replicas and publishes the scatter tables to p.tab; the segment
+// table follows in capped_segments, after the grid barrier that releases the
+// tile blocks.
+//   1. home fill, smallest home experts first (ties: lower id): each expert
+//      sums the counts of the experts filled before it in its home block;
 //   2. items (overflowing experts, overflow descending) and rooms (ranks with
-//      spare room, room descending), in one bitonic sort;
+//      spare room, room descending), compacted and sorted together;
 //   3. fillers (items below the largest room): filler f is offered to room
 //      f mod Y in round f / Y < B - 2, placed whole if it fits -- one thread
 //      per room walks its candidates;
 //   4. the stream: items not placed, cut over the rooms' space left, by
-//      prefix sums and binary searches;
-//   5. the segment table by (expert, rank): a bitonic sort of
-//      (expert, rank, piece) keys.
-__device__ void capped_build(const PlanParams &p, int T, const int *s_off, int *sm, int *s_w) {
+//      prefix sums and binary searches; the pieces, expert by expert.
+__device__ void capped_tables(const PlanParams &p, int T, const int *s_off, int *sm, int *s_w) {
   const int t = threadIdx.x;
   const int E = p.E, R = p.R, C = (int)p.SK, Bh = E / R;
   const int NP = E + R;  // bound on replica pieces (at most E + R - 1)
-  int *sT = sm;                 // [E] T_e
-  int *sh = sT + E;             // [E] h_e, pairs kept home
-  int *shb = sh + E;            // [E] home slot base of e
-  int *spb = shb + E;           // [E+1] first replica piece of e
-  int *shl = spb + E + 1;       // [E] index of e's home piece among its rank's segments
-  int *it_e = shl + E;          // [E] expert of item i (step 1: counts in fill order)
-  int *it_O = it_e + E;         // [E] overflow of item i (step 1: scan of those counts)
-  int *it_loc = it_O + E;       // [E] filler: start in its room's replica area, else -1
-  int *it_P = it_loc + E;       // [E+1] stream position of item i (step 1: home prefix)
-  int *it_s = it_P + E + 1;     // [E+1] stream index, or a filler's index in its room
-  int *it_of = it_s + E + 1;    // [E] item index of expert e, -1 if e has no overflow
-  int *st_i = it_of + E;        // [E] item at stream index s
-  int *rm_r = st_i + E;         // [R] rank of room j
-  int *rm_D = rm_r + R;         // [R] spare room
-  int *rm_left = rm_D + R;      // [R] space left after the fillers
-  int *rm_nf = rm_left + R;     // [R] fillers placed
-  int *rm_Q = rm_nf + R;        // [R] stream position of room j's space left
-  int *rm_first = rm_Q + R;     // [R] stream index of the first item meeting room j
-  int *rm_nz = rm_first + R;    // [R+1] rooms with space left before room j
-  int *rk_nh = rm_nz + R + 1;   // [R] home pieces of rank r
-  int *rk_nr = rk_nh + R;       // [R] replica pieces of rank r
-  int *pc_e = rk_nr + R;        // [NP] expert of piece
-  int *pc_r = pc_e + NP;        // [NP] rank of piece
-  int *pc_loc = pc_r + NP;      // [NP] first slot of the piece within its rank
-  int *pc_n = pc_loc + NP;      // [NP] size
-  int *pc_q = pc_n + NP;        // [NP] first overflow index of the piece within its expert
-  int *pc_li = pc_q + NP;       // [NP] index among its rank's segments (slot order)
-  uint64_t *keys = reinterpret_cast<uint64_t *>(
-      (reinterpret_cast<uintptr_t>(pc_li + NP) + 7) & ~static_cast<uintptr_t>(7));  // [n2]
-  uint32_t *skeys = reinterpret_cast<uint32_t *>(keys);  // step 5 reuses the key buffer
+  const CapMem m = cap_mem(sm, E, R);
   int tot;
 
   // ---- 1. home fill, smallest home experts first --------------------------
-  if (t < E) sT[t] = T;
+  if (t < E) {
+    m.sT[t] = T;
+    m.it_of[t] = -1;
+  }
   __syncthreads();
   const int b0 = t < E ? (t / Bh) * Bh : 0;
-  int pos = t;  // position of e in (home block, count, id) order
-  if (t < E && R > 1) {
-    int rk = 0;
-    for (int e2 = b0; e2 < b0 + Bh; ++e2) {
-      const int v = sT[e2];
-      rk += (v < T || (v == T && e2 < t)) ? 1 : 0;
+  int h = 0;
+  if (t < E) {
+    int pre = 0;  // pairs of the home experts filled before e
+    if (R > 1) {
+      for (int e2 = b0; e2 < b0 + Bh; ++e2) {
+        const int v = m.sT[e2];
+        pre += (v < T || (v == T && e2 < t)) ? v : 0;
+      }
     }
-    pos = b0 + rk;
+    // with one rank every pair fits at home
+    h = R == 1 ? T : max(0, min(T, C - pre));
+    m.sh[t] = h;
   }
-  if (t < E) it_e[pos] = T;
-  __syncthreads();
-  const int fx = block_excl_scan(t < E ? it_e[t] : 0, &tot, s_w);
-  if (t < E) it_O[t] = fx;
-  __syncthreads();
-  // with one rank every pair fits at home
-  const int h = t < E ? (R == 1 ? T : max(0, min(T, C - (it_O[pos] - it_O[b0])))) : 0;
   const int O = t < E ? T - h : 0;
-  int hf_tot;
-  const int hx = block_excl_scan(h, &tot, s_w);                  // home prefix, expert order
-  const int hf = block_excl_scan(h > 0 ? 1 : 0, &hf_tot, s_w);  // home pieces before e
-  if (t < E) {
-    it_P[t] = hx;
-    it_s[t] = hf;
-  }
-  if (t == 0) it_s[E] = hf_tot;
-  __syncthreads();
-  if (t < E) {
-    sh[t] = h;
-    shb[t] = (t / Bh) * C + (hx - it_P[b0]);
-    shl[t] = hf - it_s[b0];
-  }
-  if (t < R) rk_nh[t] = it_s[(t + 1) * Bh] - it_s[t * Bh];
   // spare room of rank t: its home load is s_off over its block
   const int Dr = t < R ? C - min(s_off[(t + 1) * Bh] - s_off[t * Bh], C) : 0;
-
-  // ---- 2. items and rooms in one sort -------------------------------------
-  int n2 = 2;
-  while (n2 < E + R) n2 <<= 1;
-  const int X = __syncthreads_count(t < E && O > 0);
-  const int Y = __syncthreads_count(t < R && Dr > 0);
-  for (int i = t; i < n2; i += kThreads) {
-    uint64_t k = ~0ull;
-    if (i < E) {
-      const int Oi = sT[i] - sh[i];
-      if (Oi > 0) k = ((uint64_t)(0x7fffffff - Oi) << 32) | (uint32_t)i;
-    } else if (i < E + R) {
-      const int r = i - E;
-      const int Dx = C - min(s_off[(r + 1) * Bh] - s_off[r * Bh], C);
-      if (Dx > 0) k = (1ull << 63) | ((uint64_t)(0x7fffffff - Dx) << 32) | (uint32_t)r;
+  __syncthreads();
+  if (t < E) {
+    int hx = 0, hn = 0;  // home pairs and home pieces of the block's experts before e
+    for (int e2 = b0; e2 < t; ++e2) {
+      const int v = m.sh[e2];
+      hx += v;
+      hn += v > 0 ? 1 : 0;
     }
-    keys[i] = k;
+    m.shb[t] = (t / Bh) * C + hx;
+    m.shl[t] = hn;
+    if (t == b0 + Bh - 1) m.rk_nh[t / Bh] = hn + (h > 0 ? 1 : 0);
   }
+
+  // ---- 2. items and rooms, compacted and sorted in one pass ----------------
+  const int isx = (t < E && O > 0) ? 1 : 0, isy = (t < R && Dr > 0) ? 1 : 0;
+  const int cpos = block_excl_scan(isx | (isy << 16), &tot, s_w);
+  const int X = tot & 0xffff, Y = tot >> 16;
+  if (isx) m.keys[cpos & 0xffff] = item_key(O, t);
+  if (isy) m.keys[X + (cpos >> 16)] = room_key(Dr, t);
   __syncthreads();
-  block_bitonic_sort(keys, n2);
-  if (t < E) it_of[t] = -1;
-  __syncthreads();
-  if (t < X) {
-    const uint64_t k = keys[t];
-    const int e = (int)(k & 0xffffffffu);
-    it_e[t] = e;
-    it_O[t] = 0x7fffffff - (int)((k >> 32) & 0x7fffffff);
-    it_of[e] = t;
-    it_loc[t] = -1;
-  }
-  if (t < Y) {
-    const uint64_t k = keys[X + t];
-    rm_r[t] = (int)(k & 0xffffffffu);
-    rm_D[t] = 0x7fffffff - (int)((k >> 32) & 0x7fffffff);
-  }
+  int n2 = 1;
+  while (n2 < X + Y) n2 <<= 1;
+  if (n2 > kThreads)
+    capped_sort_and_decode<2>(m, n2, X, Y);
+  else
+    capped_sort_and_decode<1>(m, n2, X, Y);
   __syncthreads();
 
   // ---- 3. fillers ----------------------------------------------------------
-  const int dmax = Y > 0 ? rm_D[0] : 0;
-  const int i0 = __syncthreads_count(t < X && it_O[t] >= dmax);  // items at least dmax
+  const int dmax = Y > 0 ? m.rm_D[0] : 0;
+  int i0 = 0;  // items at least dmax: the first index with it_O < dmax
+  {
+    int lo = 0, hi = X;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (m.it_O[mid] >= dmax) lo = mid + 1; else hi = mid;
+    }
+    i0 = lo;
+  }
   const int nf = X - i0;
   if (t < Y) {
-    int left = rm_D[t], cnt = 0;
+    int left = m.rm_D[t], cnt = 0;
     for (int round = 0; round < p.B - 2; ++round) {
       const int f = t + round * Y;
       if (f >= nf) break;
       const int i = i0 + f;
-      if (it_O[i] <= left) {
-        it_loc[i] = rm_D[t] - left;
-        it_s[i] = cnt;  // index among the room's fillers
-        left -= it_O[i];
+      if (m.it_O[i] <= left) {
+        m.it_loc[i] = m.rm_D[t] - left;
+        m.it_s[i] = cnt;  // index among the room's fillers
+        left -= m.it_O[i];
         ++cnt;
       }
     }
-    rm_left[t] = left;
-    rm_nf[t] = cnt;
+    m.rm_left[t] = left;
+    m.rm_nf[t] = cnt;
   }
   __syncthreads();
 
   // ---- 4. the stream -------------------------------------------------------
-  const bool ins = t < X && it_loc[t] < 0;
-  int ns_items;
-  const int P = block_excl_scan(ins ? it_O[t] : 0, &tot, s_w);
-  const int si = block_excl_scan(ins ? 1 : 0, &ns_items, s_w);
-  const int Q = block_excl_scan(t < Y ? rm_left[t] : 0, &tot, s_w);
-  const int nzx = block_excl_scan(t < Y && rm_left[t] > 0 ? 1 : 0, &tot, s_w);
+  // stream items: overflow prefix P and index; rooms: space-left prefix Q and
+  // the count of rooms with space left before (each pair packed in one scan;
+  // prefixes < 2^31, counts < 2^16)
+  const bool ins = t < X && m.it_loc[t] < 0;
+  const int left_t = t < Y ? m.rm_left[t] : 0;
+  long long tot64;
+  const long long pq = block_excl_scan64(
+      (long long)(ins ? m.it_O[t] : 0) | ((long long)left_t << 32), &tot64);
+  const int cnts = block_excl_scan((ins ? 1 : 0) | ((left_t > 0 ? 1 : 0) << 16), &tot, s_w);
+  const int ns_items = tot & 0xffff;
   if (ins) {
-    it_P[t] = P;
-    it_s[t] = si;
-    st_i[si] = t;
+    m.it_P[t] = (int)(pq & 0xffffffffll);
+    m.it_s[t] = cnts & 0xffff;
+    m.st_i[cnts & 0xffff] = t;
   }
   if (t < Y) {
-    rm_Q[t] = Q;
-    rm_nz[t] = nzx;
+    m.rm_Q[t] = (int)(pq >> 32);
+    m.rm_nz[t] = cnts >> 16;
   }
-  if (t == 0) rm_nz[Y] = tot;
+  if (t == 0) m.rm_nz[Y] = tot >> 16;
   __syncthreads();
-  // stream index of the first item meeting room j
-  if (t < Y && rm_left[t] > 0) {
-    int lo = 0, hi = ns_items;  // last s with P(st_i[s]) <= Q
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if (it_P[st_i[mid]] <= rm_Q[t]) lo = mid; else hi = mid;
+  // stream index of the first item meeting room j, and the stream items that
+  // meet it
+  int nrep_j = 0;
+  if (t < Y) {
+    int nst = 0;
+    if (m.rm_left[t] > 0) {
+      int lo = 0, hi = ns_items;  // last s with P(st_i[s]) <= Q
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (m.it_P[m.st_i[mid]] <= m.rm_Q[t]) lo = mid; else hi = mid;
+      }
+      m.rm_first[t] = lo;
+      int lo2 = lo, hi2 = ns_items;  // last s with P(st_i[s]) <= Q + left - 1
+      const int last = m.rm_Q[t] + m.rm_left[t] - 1;
+      while (hi2 - lo2 > 1) {
+        const int mid = (lo2 + hi2) >> 1;
+        if (m.it_P[m.st_i[mid]] <= last) lo2 = mid; else hi2 = mid;
+      }
+      nst = lo2 - lo + 1;
     }
-    rm_first[t] = lo;
+    nrep_j = m.rm_nf[t] + nst;
   }
   __syncthreads();
   // pieces of expert t: its filler, or its stream pieces
   int npc = 0, j0 = 0, j1 = -1;
-  const int it = t < E ? it_of[t] : -1;
+  const int it = t < E ? m.it_of[t] : -1;
   if (it >= 0) {
-    if (it_loc[it] >= 0) {
+    if (m.it_loc[it] >= 0) {
       npc = 1;
     } else {
-      const int a = it_P[it], b = a + it_O[it];
-      j0 = last_le(rm_Q, Y, a);
-      j1 = last_le(rm_Q, Y, b - 1);
-      npc = rm_nz[j1 + 1] - rm_nz[j0];
+      const int a = m.it_P[it], b = a + m.it_O[it];
+      j0 = last_le(m.rm_Q, Y, a);
+      j1 = last_le(m.rm_Q, Y, b - 1);
+      npc = m.rm_nz[j1 + 1] - m.rm_nz[j0];
     }
   }
-  int npieces;
-  const int pb = block_excl_scan(npc, &npieces, s_w);
-  if (t < E) spb[t] = pb;
-  if (t == 0) spb[E] = npieces;
-  __syncthreads();
+  // replica pieces before e, and home pieces before e (both < 2^16)
+  const int pc = block_excl_scan(npc | ((t < E && h > 0 ? 1 : 0) << 16), &tot, s_w);
+  const int pb = pc & 0xffff, npieces = tot & 0xffff;
+  if (t < E) {
+    m.spb[t] = pb;
+    m.shf[t] = pc >> 16;
+  }
+  if (t == 0) {
+    m.spb[E] = npieces;
+    m.misc[0] = tot >> 16;  // home pieces
+    m.misc[1] = npieces;
+  }
+  if (t < R) m.rk_nr[t] = 0;
   if (it >= 0 && pb + npc <= NP) {  // at most E + R - 1 pieces by construction
     const int e = t;
-    if (it_loc[it] >= 0) {
+    if (m.it_loc[it] >= 0) {
       const int j = (it - i0) % Y;
-      const int r = rm_r[j];
-      pc_e[pb] = e;
-      pc_r[pb] = r;
-      pc_loc[pb] = (C - rm_D[j]) + it_loc[it];
-      pc_n[pb] = it_O[it];
-      pc_q[pb] = 0;
-      pc_li[pb] = rk_nh[r] + it_s[it];
+      const int r = m.rm_r[j];
+      m.pc_e[pb] = e;
+      m.pc_r[pb] = r;
+      m.pc_loc[pb] = (C - m.rm_D[j]) + m.it_loc[it];
+      m.pc_n[pb] = m.it_O[it];
+      m.pc_q[pb] = 0;
+      m.pc_li[pb] = m.rk_nh[r] + m.it_s[it];
     } else {
-      const int a = it_P[it], b = a + it_O[it];
+      const int a = m.it_P[it], b = a + m.it_O[it];
       int q = pb;
       for (int j = j0; j <= j1; ++j) {
-        if (rm_left[j] == 0) continue;
-        const int r = rm_r[j];
-        const int lo = max(a, rm_Q[j]), hi = min(b, rm_Q[j] + rm_left[j]);
-        pc_e[q] = e;
-        pc_r[q] = r;
-        pc_loc[q] = (C - rm_D[j]) + (rm_D[j] - rm_left[j]) + (lo - rm_Q[j]);
-        pc_n[q] = hi - lo;
-        pc_q[q] = lo - a;
-        pc_li[q] = rk_nh[r] + rm_nf[j] + (it_s[it] - rm_first[j]);
+        if (m.rm_left[j] == 0) continue;
+        const int r = m.rm_r[j];
+        const int lo = max(a, m.rm_Q[j]), hi = min(b, m.rm_Q[j] + m.rm_left[j]);
+        m.pc_e[q] = e;
+        m.pc_r[q] = r;
+        m.pc_loc[q] = (C - m.rm_D[j]) + (m.rm_D[j] - m.rm_left[j]) + (lo - m.rm_Q[j]);
+        m.pc_n[q] = hi - lo;
+        m.pc_q[q] = lo - a;
+        m.pc_li[q] = m.rk_nh[r] + m.rm_nf[j] + (m.it_s[it] - m.rm_first[j]);
         ++q;
       }
     }
   }
-  // replica pieces per rank: fillers plus the stream items meeting the room
-  if (t < R) rk_nr[t] = 0;
   __syncthreads();
-  int nrep_j = 0;
-  if (t < Y) {
-    int nst = 0;
-    if (rm_left[t] > 0) {
-      int lo = 0, hi = ns_items;  // last s with P(st_i[s]) <= Q + left - 1
-      const int last = rm_Q[t] + rm_left[t] - 1;
-      while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (it_P[st_i[mid]] <= last) lo = mid; else hi = mid;
-      }
-      nst = lo - rm_first[t] + 1;
-    }
-    nrep_j = rm_nf[t] + nst;
-    rk_nr[rm_r[t]] = nrep_j;
-  }
+  if (t < Y) m.rk_nr[m.rm_r[t]] = nrep_j;
   const int mx = block_max(nrep_j, s_w);  // syncs
+  if (t == 0 && p.max_rank_replicas != nullptr) *p.max_rank_replicas = mx;
   // publish the scatter tables
   int *tab_h = p.tab, *tab_hb = tab_h + E, *tab_pb = tab_hb + E;
   int *tab_pq = tab_pb + E + 1, *tab_pbase = tab_pq + NP;
   if (t < E) {
-    __stcg(tab_h + t, sh[t]);
-    __stcg(tab_hb + t, shb[t]);
-    __stcg(tab_pb + t, spb[t]);
+    __stcg(tab_h + t, m.sh[t]);
+    __stcg(tab_hb + t, m.shb[t]);
+    __stcg(tab_pb + t, pb);
   }
-  if (t == 0) __stcg(tab_pb + E, spb[E]);
+  if (t == 0) __stcg(tab_pb + E, npieces);
   for (int q = t; q < npieces; q += kThreads) {
-    __stcg(tab_pq + q, pc_q[q]);
-    __stcg(tab_pbase + q, pc_r[q] * C + pc_loc[q] - pc_q[q]);
+    __stcg(tab_pq + q, m.pc_q[q]);
+    __stcg(tab_pbase + q, m.pc_r[q] * C + m.pc_loc[q] - m.pc_q[q]);
   }
+}
 
-  // ---- 5. the segment table, by (expert, rank) -----------------------------
-  const int nhome = it_s[E];
-  const int nseg = nhome + npieces;
-  int m2 = 2;
-  while (m2 < nseg) m2 <<= 1;
-  // keys: expert (bits 21..30), rank (11..20), piece id (0..10; 2047 = home)
-  for (int i = t; i < m2; i += kThreads) skeys[i] = 0xffffffffu;
-  __syncthreads();
-  if (t < E && h > 0) skeys[hf] = ((uint32_t)t << 21) | ((uint32_t)(t / Bh) << 11) | 2047u;
-  for (int q = t; q < npieces; q += kThreads)
-    skeys[nhome + q] = ((uint32_t)pc_e[q] << 21) | ((uint32_t)pc_r[q] << 11) | (uint32_t)q;
-  __syncthreads();
-  block_bitonic_sort(skeys, m2);
-  // rank_seg_ptr: each rank's home and replica segments
+// The capped plan's segment table, by (expert, rank), from the builder's
+// arrays (the coordinator, after the tables are published).  An expert's
+// segments are its home piece and its replica pieces in rank order; a
+// piece's place among them is the number of the expert's pieces on lower
+// ranks.  Also writes rank_seg_ptr, rank_seg_idx, replica_seg,
+// expert_seg_ptr, num_seg and num_replicas.
+__device__ void capped_segments(const PlanParams &p, int *sm, int *s_w) {
+  const int t = threadIdx.x;
+  const int E = p.E, R = p.R, C = (int)p.SK, Bh = E / R;
+  const CapMem m = cap_mem(sm, E, R);
+  const int nhome = m.misc[0], npieces = m.misc[1];
   int rtot;
-  const int rsp = block_excl_scan(t < R ? rk_nh[t] + rk_nr[t] : 0, &rtot, s_w);
+  const int rsp = block_excl_scan(t < R ? m.rk_nh[t] + m.rk_nr[t] : 0, &rtot, s_w);
   if (t < R) {
     p.rank_seg_ptr[t] = rsp;
-    rm_Q[t] = rsp;  // rank_seg_ptr, kept for the writes below (rm_Q is no longer needed)
+    m.rm_Q[t] = rsp;  // rank_seg_ptr (rm_Q is no longer needed)
   }
   if (t == 0) p.rank_seg_ptr[R] = rtot;
   __syncthreads();
-  // segments a = 2t and 2t + 1 of the table (at most 2047 of them)
-  bool rep[2];
-#pragma unroll
-  for (int u = 0; u < 2; ++u) {
-    const int a = 2 * t + u;
-    rep[u] = false;
-    if (a < nseg) {
-      const uint32_t k = skeys[a];
-      rep[u] = (int)((k >> 11) & 1023u) != (int)(k >> 21) / Bh;
+  const int lim = E + R - 1;  // rank_seg_idx entries
+  for (int e = t; e < E; e += kThreads) {
+    const int b = m.spb[e], n = m.spb[e + 1] - b;
+    const int base = m.shf[e] + b;  // segments of the experts before e
+    p.expert_seg_ptr[e] = base;
+    const int h = m.sh[e];
+    if (h > 0) {
+      const int home = e / Bh;
+      int lower = 0;
+      for (int q = b; q < b + n; ++q) lower += m.pc_r[q] < home ? 1 : 0;
+      const int a = base + lower;
+      p.seg[a] = make_int4(e, home, m.shb[e] - home * C, h);
+      const int at = m.rm_Q[home] + m.shl[e];
+      if (at >= 0 && at < lim) p.rank_seg_idx[at] = a;
     }
   }
-  int nrep_tot;
-  int rpos = block_excl_scan((rep[0] ? 1 : 0) + (rep[1] ? 1 : 0), &nrep_tot, s_w);
-#pragma unroll
-  for (int u = 0; u < 2; ++u) {
-    const int a = 2 * t + u;
-    if (a >= nseg) continue;
-    const uint32_t k = skeys[a];
-    const int e = (int)(k >> 21), r = (int)((k >> 11) & 1023u), pid = (int)(k & 2047u);
-    int start, cnt, li;
-    if (pid == 2047) {
-      start = shb[e] - r * C;
-      cnt = sh[e];
-      li = shl[e];
-    } else {
-      start = pc_loc[pid];
-      cnt = pc_n[pid];
-      li = pc_li[pid];
-    }
-    p.seg[a] = make_int4(e, r, start, cnt);
-    const int at = rm_Q[r] + li;
-    if (at >= 0 && at < E + R - 1) p.rank_seg_idx[at] = a;
-    if (rep[u]) p.replica_seg[rpos++] = a;
-  }
-  // first segment of each expert (the first key at or above e << 21)
-  for (int e = t; e <= E; e += kThreads) {
-    int lo = 0, hi = nseg;
-    const uint32_t want = (uint32_t)e << 21;
-    while (lo < hi) {
-      const int mid = (lo + hi) >> 1;
-      if (skeys[mid] < want) lo = mid + 1; else hi = mid;
-    }
-    p.expert_seg_ptr[e] = lo;
+  for (int q = t; q < npieces; q += kThreads) {
+    const int e = m.pc_e[q], r = m.pc_r[q];
+    const int b = m.spb[e], n = m.spb[e + 1] - b;
+    int lower = 0;
+    for (int q2 = b; q2 < b + n; ++q2) lower += m.pc_r[q2] < r ? 1 : 0;
+    const int a = m.shf[e] + b + lower + ((m.sh[e] > 0 && e / Bh < r) ? 1 : 0);
+    p.seg[a] = make_int4(e, r, m.pc_loc[q], m.pc_n[q]);
+    const int at = m.rm_Q[r] + m.pc_li[q];
+    if (at >= 0 && at < lim) p.rank_seg_idx[at] = a;
+    p.replica_seg[b + lower] = a;  // replicas in table order
   }
   if (t == 0) {
-    *p.num_seg = nseg;
-    *p.num_replicas = nrep_tot;
-    if (p.max_rank_replicas != nullptr) *p.max_rank_replicas = mx;
+    p.expert_seg_ptr[E] = nhome + npieces;
+    *p.num_seg = nhome + npieces;
+    *p.num_replicas = npieces;
   }
 }
 
@@ -932,19 +1067,62 @@ __global__ void __launch_bounds__(kThreads, 1) plan_kernel(PlanParams p) {
     } else {  // kPlanCapped: the coordinator (never a tile block) builds the tables
       if (t < E) p.expert_offset[t] = off;
       if (t == 0) p.expert_offset[E] = total;
-      capped_build(p, T, s_off, smem, s_w);
+      capped_tables(p, T, s_off, smem, s_w);
     }
   }
 
-  // The capped plan's tables reach the tile blocks through the workspace,
-  // after one more grid barrier: per expert h_e, its home slot base and its
-  // first piece; per piece its first overflow index and slot base.
+  // The capped plan's slots come in two passes around one more grid barrier:
+  // before it, while the coordinator builds its tables, the tile blocks give
+  // each pair its position in the expert-sorted order (kept in slot); after
+  // it they turn that position into the slot through the published tables
+  // (per expert h_e, its home slot base and first piece; per piece its first
+  // overflow index and slot base) while the coordinator writes the segments.
   const bool cap = p.full && p.kind == kPlanCapped;
-  int *s_ch = s_tab[1], *s_chb = s_tab[2], *s_cpb = s_tab[3];
-  int *s_cpq = &s_tab[4][0], *s_cpbase = &s_tab[4][0] + 2 * kTab;
+  const unsigned nk = (unsigned)p.NK;
+  int32_t *slot_w = p.slot + p.pair0 + w0;
+  const int q0 = (int)(p.pair0 + w0);  // global pair index of the warp's first pair
+  if (p.full && !coord) {
+    // Per expert: where this tile's pairs start in the expert-sorted order
+    // (expert offset + tile offset); wh keeps the warp offsets in the tile.
+    int *s_base = s_tab[7];
+    __syncthreads();  // a single block has finished the coordinator's tables
+    if (t < E) s_base[t] = off + tile_off;
+    __syncthreads();
+
+    const bool hf = p.kind == kPlanHomeFirst;
+    const unsigned lt = lanemask_lt(), gt = lanemask_gt();
+    for (int c = 0; c < nw; c += 32) {
+      const int i = c + lane;
+      const bool act = i < nw;
+      int e = -1;
+      if (act) e = keep ? ids[i] : __ldg(idx_w + i);
+      const bool valid = (unsigned)e < (unsigned)E;
+      const unsigned peers = peers_of(valid ? e : sentinel, nbits);
+      const int wo = valid ? wh[e] : 0;
+      __syncwarp();
+      if (valid) {
+        // rank among the tile's pairs of e -- one population count per step:
+        // bit counts and leading-one searches go to the narrow XU pipe, which
+        // the profile showed as this loop's busiest unit
+        const int r = wo + __popc(peers & lt);
+        int s = s_base[e] + r;  // position in the expert-sorted order
+        if (hf) s = home_first_slot(e, s - s_off[e], Bx, C, p.R, s_h, s_off, s_O, s_F, s_D, s_rf);
+        slot_w[i] = s;
+        if (!cap && (unsigned)s < nk) p.src_pair[s] = q0 + i;
+        if ((peers & gt) == 0) wh[e] = r + 1;  // the last of the peers moves the cursor
+      } else if (act) {
+        slot_w[i] = -1;
+      }
+      __syncwarp();
+    }
+  }
   if (cap) {
     if (!plan_sync(p, direct ? 2 : 3)) return;
-    if (!coord) {
+    if (coord) {
+      capped_segments(p, smem, s_w);
+    } else {
+      int *s_ch = s_tab[1], *s_chb = s_tab[2], *s_cpb = s_tab[3];
+      int *s_cpq = &s_tab[4][0], *s_cpbase = &s_tab[4][0] + 2 * kTab;
       const int *tab_h = p.tab, *tab_hb = tab_h + E, *tab_pb = tab_hb + E;
       const int *tab_pq = tab_pb + E + 1, *tab_pbase = tab_pq + (E + p.R);
       const int npieces = min(__ldcg(tab_pb + E), 2 * kTab);
@@ -958,43 +1136,29 @@ __global__ void __launch_bounds__(kThreads, 1) plan_kernel(PlanParams p) {
         s_cpq[i] = __ldcg(tab_pq + i);
         s_cpbase[i] = __ldcg(tab_pbase + i);
       }
-    }
-  }
-
-  if (p.full && !coord) {
-    // Per expert: where this tile's pairs start in the expert-sorted order
-    // (expert offset + tile offset); wh keeps the warp offsets in the tile.
-    int *s_base = cap ? s_rank : s_tab[7];
-    __syncthreads();  // a single block has finished the coordinator's tables
-    if (t < E) s_base[t] = off + tile_off;
-    __syncthreads();
-
-    const bool hf = p.kind == kPlanHomeFirst;
-    const unsigned lt = lanemask_lt();
-    const unsigned nk = (unsigned)p.NK;
-    int32_t *slot_w = p.slot + p.pair0 + w0;
-    const int q0 = (int)(p.pair0 + w0);  // global pair index of the warp's first pair
-    for (int c = 0; c < nw; c += 32) {
-      const int i = c + lane;
-      const bool act = i < nw;
-      int e = -1;
-      if (act) e = keep ? ids[i] : __ldg(idx_w + i);
-      const bool valid = (unsigned)e < (unsigned)E;
-      const unsigned peers = peers_of(valid ? e : sentinel, nbits);
-      const int wo = valid ? wh[e] : 0;
-      __syncwarp();
-      if (valid) {
-        const int r = wo + __popc(peers & lt);  // rank among the tile's pairs of e
-        int s = s_base[e] + r;                  // position in the expert-sorted order
-        if (hf) s = home_first_slot(e, s - s_off[e], Bx, C, p.R, s_h, s_off, s_O, s_F, s_D, s_rf);
-        if (cap) s = capped_slot(e, s - s_off[e], s_ch, s_chb, s_cpb, s_cpq, s_cpbase);
-        slot_w[i] = s;
-        if ((unsigned)s < nk) p.src_pair[s] = q0 + i;
-        if (lane == __ffs(peers) - 1) wh[e] = wo + __popc(peers);
-      } else if (act) {
-        slot_w[i] = -1;
+      __syncthreads();
+      for (int c = 0; c < nw; c += 32 * kBatch) {
+        int sv[kBatch], ev[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {  // all loads in flight together
+          const int i = c + u * 32 + lane;
+          sv[u] = -1;
+          ev[u] = 0;
+          if (i < nw) {
+            sv[u] = slot_w[i];
+            ev[u] = keep ? ids[i] : __ldg(idx_w + i);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+          if (sv[u] < 0) continue;  // an id out of range (slot -1)
+          const int i = c + u * 32 + lane;
+          const int e = ev[u];
+          const int s = capped_slot(e, sv[u] - s_off[e], s_ch, s_chb, s_cpb, s_cpq, s_cpbase);
+          slot_w[i] = s;
+          if ((unsigned)s < nk) p.src_pair[s] = q0 + i;
+        }
       }
-      __syncwarp();
     }
   }
   if (p.nb > 1) grid_barrier_exit(p.bar, p.nb);
@@ -1064,10 +1228,13 @@ cudaError_t launch_plan(const mep_shape_t &s, const int32_t *idx, const mep_plan
   if (capped) {
     cap = std::min<int64_t>(cap, kPlanMaxBlocks - kPlanCappedTabRows);
     if (cap < 1) return cudaErrorInvalidConfiguration;
-    if (capped_tab_words(s.E, s.R) > (int64_t)s.E * kPlanCappedTabRows) return cudaErrorInvalidValue;
+    if (capped_tab_words(s.E, s.R) > (int64_t)s.E * kPlanCappedTabRows ||
+        capped_smem_ints(s.E, s.R) > (int64_t)kWarps * (s.E + kPlanIdsPerWarp))
+      return cudaErrorInvalidValue;
   }
   const int nt = (int)std::max<int64_t>(1, std::min<int64_t>(want, cap));
   const int nb = (nt > 1 || capped) ? nt + 1 : 1;
+  const int64_t ppb = (NKt + nt - 1) / nt;
   PlanParams p{};
   p.idx = idx;
   p.R = s.R; p.S = s.S; p.E = s.E; p.K = s.K;
@@ -1075,7 +1242,7 @@ cudaError_t launch_plan(const mep_shape_t &s, const int32_t *idx, const mep_plan
   p.SK = (int64_t)s.S * s.K;
   p.nb = nb;
   p.nt = nt;
-  p.ppb = (NKt + nt - 1) / nt;
+  p.ppb = ppb;
   p.NKt = NKt;
   p.pair0 = ranked ? (int64_t)x.rank * s.S * s.K : 0;
   p.rank_counts = x.rank_counts;
