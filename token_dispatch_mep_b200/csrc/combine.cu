@@ -74,9 +74,6 @@
 #ifndef MEP_COMBINE_CVT
 #define MEP_COMBINE_CVT 0  // 1: bf16 -> float32 -> binary64 by conversion instructions
 #endif
-#ifndef MEP_COMBINE_PERSIST
-#define MEP_COMBINE_PERSIST 0  // 1: resident grid; each warp loads its next token's ids early
-#endif
 
 namespace mep {
 
@@ -210,25 +207,9 @@ __global__ void __launch_bounds__(kThreads, MEP_COMBINE_MIN_BLOCKS) combine_row_
   const int lane = threadIdx.x & 31;
   const int64_t nwarps = (int64_t)gridDim.x * kWarps;
   bool bad = false;
-  int64_t g = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
-#if MEP_COMBINE_PERSIST
-  // the next token's slot ids and weights are loaded one token ahead
-  int sl_next = (g < p.N && lane < p.K) ? __ldg(p.slot + (p.g0 + g) * p.K + lane) : -1;
-  float wt_next = (g < p.N && lane < p.K) ? (p.w != nullptr ? __ldg(p.w + g * p.K + lane) : 1.f) : 0.f;
-#endif
-  for (; g < p.N; g += nwarps) {
-#if MEP_COMBINE_PERSIST
-    int sl = sl_next;
-    const float wt = wt_next;
-    {
-      const int64_t gn = g + nwarps;
-      sl_next = (gn < p.N && lane < p.K) ? __ldg(p.slot + (p.g0 + gn) * p.K + lane) : -1;
-      wt_next = (gn < p.N && lane < p.K) ? (p.w != nullptr ? __ldg(p.w + gn * p.K + lane) : 1.f) : 0.f;
-    }
-#else
+  for (int64_t g = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5); g < p.N; g += nwarps) {
     int sl = lane < p.K ? __ldg(p.slot + (p.g0 + g) * p.K + lane) : -1;
     const float wt = lane < p.K ? (p.w != nullptr ? __ldg(p.w + g * p.K + lane) : 1.f) : 0.f;
-#endif
     if (lane < p.K && (unsigned)sl >= (unsigned)p.NK) {
       bad = true;
       sl = -1;
@@ -308,11 +289,7 @@ __global__ void __launch_bounds__(kThreads, MEP_COMBINE_MIN_BLOCKS) combine_row_
 template <int KC>
 cudaError_t launch_kc(const CombineParams &p, int sms, cudaStream_t stream) {
   const int64_t want = (p.N + kWarps - 1) / kWarps;
-#if MEP_COMBINE_PERSIST
-  const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>(want, (int64_t)sms * MEP_COMBINE_MIN_BLOCKS));
-#else
   const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>(want, (int64_t)sms * 1024));
-#endif
   if (p.rank_ys != nullptr)
     return launch_pdl(combine_row_kernel<KC, true>, dim3(blocks), dim3(kThreads), 0, stream, p);
   return launch_pdl(combine_row_kernel<KC, false>, dim3(blocks), dim3(kThreads), 0, stream, p);
