@@ -247,42 +247,28 @@ __device__ __forceinline__ Key bitonic_keep(Key x, Key y, int i, int j, int k) {
   return keep_min == lt ? x : y;
 }
 
-// Ascending bitonic sort of n2 keys (n2 a power of two, n2 <= V * blockDim.x)
-// held in registers: thread t holds positions t and t + blockDim.x.  Steps
-// with a partner inside the warp exchange by shuffle; longer ones go through
-// shared memory (buf: 2 * n2 keys, double-buffered, one barrier per step);
-// with V = 2 the longest step pairs a thread's own two keys.  Every thread of
-// the block calls it; positions >= n2 are ignored.
-template <typename Key, int V>
-__device__ void block_sort_regs(Key (&x)[V], int n2, Key *buf) {
+// Ascending bitonic sort of n2 keys (n2 a power of two, n2 <= blockDim.x)
+// held in registers, one per thread (position = thread index).  Steps with a
+// partner inside the warp exchange by shuffle; longer ones go through shared
+// memory (buf: 2 * n2 keys, double-buffered, one barrier per step).  Every
+// thread of the block calls it; positions >= n2 are ignored.
+template <typename Key>
+__device__ void block_sort_regs(Key &x, int n2, Key *buf) {
   const int t = threadIdx.x;
   int cur = 0;
   for (int k = 2; k <= n2; k <<= 1) {
     for (int j = k >> 1; j > 0; j >>= 1) {
-      Key y[V];
-      if (j >= kThreads) {  // only with V == 2: positions t and t + kThreads
-        y[0] = x[V - 1];
-        y[V - 1] = x[0];
-      } else if (j >= 32) {
+      Key y;
+      if (j >= 32) {
         Key *b = buf + cur * n2;
-#pragma unroll
-        for (int u = 0; u < V; ++u) {
-          const int i = t + u * kThreads;
-          if (i < n2) b[i] = x[u];
-        }
+        if (t < n2) b[t] = x;
         __syncthreads();
-#pragma unroll
-        for (int u = 0; u < V; ++u) {
-          const int i = t + u * kThreads;
-          y[u] = i < n2 ? b[i ^ j] : x[u];
-        }
+        y = t < n2 ? b[t ^ j] : x;
         cur ^= 1;
       } else {
-#pragma unroll
-        for (int u = 0; u < V; ++u) y[u] = __shfl_xor_sync(0xffffffffu, x[u], j);
+        y = __shfl_xor_sync(0xffffffffu, x, j);
       }
-#pragma unroll
-      for (int u = 0; u < V; ++u) x[u] = bitonic_keep(x[u], y[u], t + u * kThreads, j, k);
+      x = bitonic_keep(x, y, t, j, k);
     }
   }
 }
@@ -302,12 +288,12 @@ __host__ __device__ __forceinline__ int64_t capped_tab_words(int E, int R) {
 
 // Shared-memory ints the capped builder uses: 13 E + 9 R + 6 (E + R) + 8,
 // plus two sort buffers of n2 8-byte keys (n2 the power of two at or above
-// the items and rooms, at most E + R).  The coordinator's dynamic shared
+// the items and rooms, who number at most E).  The coordinator's dynamic shared
 // memory holds kWarps * (E + kPlanIdsPerWarp) ints, which is more for every
 // E <= MEP_MAX_EXPERTS (R <= E); the launch checks it.
 __host__ __device__ __forceinline__ int64_t capped_smem_ints(int E, int R) {
-  int64_t n2 = 1;  // sort size bound: the power of two at or above E + R
-  while (n2 < (int64_t)E + R) n2 <<= 1;
+  int64_t n2 = 1;  // sort size bound: the power of two at or above E (items + rooms <= E)
+  while (n2 < (int64_t)E) n2 <<= 1;
   return 13 * (int64_t)E + 9 * (int64_t)R + 6 * ((int64_t)E + R) + 8 + 4 * n2;
 }
 
@@ -371,7 +357,7 @@ __device__ __forceinline__ CapMem cap_mem(int *sm, int E, int R) {
   m.rk_nr = q; q += R;
   m.misc = q; q += 4;
   q = reinterpret_cast<int *>((reinterpret_cast<uintptr_t>(q) + 7) & ~static_cast<uintptr_t>(7));
-  m.keys = reinterpret_cast<uint64_t *>(q);  // n2 <= 2 NP - 1 keys: inside the 6 NP piece ints
+  m.keys = reinterpret_cast<uint64_t *>(q);  // X + Y <= E keys: inside the 6 NP piece ints
   m.pc_e = q; q += NP;
   m.pc_r = q; q += NP;
   m.pc_loc = q; q += NP;
@@ -392,30 +378,22 @@ __device__ __forceinline__ uint64_t room_key(int D, int r) {
   return (1ull << 63) | ((uint64_t)(0x7fffffff - D) << 32) | (uint32_t)r;
 }
 
-template <int V>
+// Sorts the X items and Y rooms of keys[0, X + Y) (n2 >= X + Y, n2 <=
+// blockDim.x) and writes the item and room tables.
 __device__ __forceinline__ void capped_sort_and_decode(const CapMem &m, int n2, int X, int Y) {
   const int t = threadIdx.x;
-  uint64_t x[V];
-#pragma unroll
-  for (int u = 0; u < V; ++u) {
-    const int i = t + u * kThreads;
-    x[u] = i < X + Y ? m.keys[i] : ~0ull;
-  }
-  block_sort_regs<uint64_t, V>(x, n2, m.sbuf);
-#pragma unroll
-  for (int u = 0; u < V; ++u) {
-    const int i = t + u * kThreads;
-    const int id = (int)(x[u] & 0xffffffffu);
-    const int v = 0x7fffffff - (int)((x[u] >> 32) & 0x7fffffff);
-    if (i < X) {
-      m.it_e[i] = id;
-      m.it_O[i] = v;
-      m.it_of[id] = i;
-      m.it_loc[i] = -1;
-    } else if (i < X + Y) {
-      m.rm_r[i - X] = id;
-      m.rm_D[i - X] = v;
-    }
+  uint64_t x = t < X + Y ? m.keys[t] : ~0ull;
+  block_sort_regs<uint64_t>(x, n2, m.sbuf);
+  const int id = (int)(x & 0xffffffffu);
+  const int v = 0x7fffffff - (int)((x >> 32) & 0x7fffffff);
+  if (t < X) {
+    m.it_e[t] = id;
+    m.it_O[t] = v;
+    m.it_of[id] = t;
+    m.it_loc[t] = -1;
+  } else if (t < X + Y) {
+    m.rm_r[t - X] = id;
+    m.rm_D[t - X] = v;
   }
 }
 
@@ -484,12 +462,16 @@ __device__ void capped_tables(const PlanParams &p, int T, const int *s_off, int 
   if (isx) m.keys[cpos & 0xffff] = item_key(O, t);
   if (isy) m.keys[X + (cpos >> 16)] = room_key(Dr, t);
   __syncthreads();
+  // X + Y <= E <= kThreads: an overflowing expert's home rank is full, so the
+  // items come from full ranks (E/R experts each) and the rooms are the
+  // other ranks -- X + Y <= (E/R) F + (R - F) <= E for F full ranks.
   int n2 = 1;
   while (n2 < X + Y) n2 <<= 1;
-  if (n2 > kThreads)
-    capped_sort_and_decode<2>(m, n2, X, Y);
-  else
-    capped_sort_and_decode<1>(m, n2, X, Y);
+  if (n2 > kThreads) {  // unreachable by the bound above; never sorted partially
+    if (t == 0) set_status(p.status, MEP_ERR_DEVICE_DATA);
+    n2 = kThreads;
+  }
+  capped_sort_and_decode(m, n2, min(X, kThreads), min(Y, kThreads - min(X, kThreads)));
   __syncthreads();
 
   // ---- 3. fillers ----------------------------------------------------------
