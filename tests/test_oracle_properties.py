@@ -77,6 +77,28 @@ def test_capped_plan_is_the_queue_simulation(case, B):
 
 
 @SETTINGS
+@given(routed(), st.integers(1, 8))
+def test_capped_items_and_rooms_number_at_most_E(case, B):
+    """The capped schedule's items (experts that overflow their home rank)
+    and rooms (ranks with spare room after their home fill) number at most E
+    together: an overflowing expert's home rank is full, so items come from
+    full ranks (E/R experts each) and rooms are the other ranks.  The GPU
+    builder sorts them with one key per thread of a 1024-thread block and
+    relies on this bound (E <= 1024)."""
+    R, S, E, K, idx = case
+    pl = ORA.plan_capped(R, S, E, K, B, idx)
+    C, Bh = S * K, E // R
+    counts = np.bincount(idx.ravel(), minlength=E)
+    seg = pl["seg"][:pl["num_seg"]]
+    items = {int(e) for e, r, _, _ in seg if r != e // Bh}   # experts with a replica piece
+    home_load = counts.reshape(R, Bh).sum(axis=1)
+    rooms = int((home_load < C).sum())
+    assert len(items) + rooms <= E
+    full = int((home_load >= C).sum())
+    assert len(items) <= Bh * full
+
+
+@SETTINGS
 @given(routed(), st.integers(1, 5), st.integers(0, 2 ** 31 - 1))
 def test_combine_and_reduce_are_exact_sums(case, P, seed):
     R, S, E, K, idx = case
