@@ -36,7 +36,13 @@
 // warp broadcasts with shuffles.  The K expert-output chunks are loaded in
 // groups of 8 (all loads of a group issued before any use) and accumulated in
 // k order; the sum is rounded to bf16 and written with a streaming 16-byte
-// store.  Expert outputs are read once (streaming loads).  The grid has one
+// store.  Expert outputs are read once (streaming loads).  The kernel is
+// instantiated for K up to 2, 4, 6, 8 and 16 terms: a warp's loads in flight
+// are held in registers, so an instantiation no wider than K leaves room for
+// more resident warps (for K = 6: a launch bound of 9 blocks per SM, which
+// the compiler meets with 96 registers -- 10 resident blocks, against 8 for
+// the K = 8 form -- measured 0.96 of the copy peak against 0.92; bounds of 8
+// and 10 measured 0.93 and 0.95).  The grid has one
 // warp per token, in blocks of two warps: small blocks keep the last wave
 // short (1 % over blocks of eight warps).  A form with warp tasks over parts
 // of rows and all K loads in flight measured 0.90-1.00 of the HBM copy peak
@@ -61,6 +67,12 @@
 
 #ifndef MEP_COMBINE_MIN_BLOCKS
 #define MEP_COMBINE_MIN_BLOCKS 8  // launch bound: resident blocks per SM
+#endif
+#ifndef MEP_COMBINE_K6
+#define MEP_COMBINE_K6 1  // 1: a K <= 6 instantiation (loads and registers for 6 terms)
+#endif
+#ifndef MEP_COMBINE_MIN_BLOCKS_K6
+#define MEP_COMBINE_MIN_BLOCKS_K6 9  // its launch bound (blocks per SM)
 #endif
 #ifndef MEP_COMBINE_ROW_U
 #define MEP_COMBINE_ROW_U 2  // 16-byte chunks per lane per step
@@ -200,7 +212,8 @@ __device__ __forceinline__ const uint16_t *slot_row(const CombineParams &p, int6
 }
 
 template <int KC, bool kRanked>
-__global__ void __launch_bounds__(kThreads, MEP_COMBINE_MIN_BLOCKS) combine_row_kernel(CombineParams p) {
+__global__ void __launch_bounds__(kThreads, KC == 6 ? MEP_COMBINE_MIN_BLOCKS_K6 : MEP_COMBINE_MIN_BLOCKS)
+    combine_row_kernel(CombineParams p) {
   griddep_wait();  // the previous kernel on the stream is complete and visible
   constexpr int KG = KC < MEP_COMBINE_GROUP ? KC : MEP_COMBINE_GROUP;
   constexpr int kRU = MEP_COMBINE_ROW_U;
@@ -322,6 +335,9 @@ cudaError_t launch_combine(const mep_shape_t &s, int32_t H, const mep_plan_t &pl
   p.chunks = H / 8;
   if (s.K <= 2) return launch_kc<2>(p, sms, stream);
   if (s.K <= 4) return launch_kc<4>(p, sms, stream);
+#if MEP_COMBINE_K6
+  if (s.K <= 6) return launch_kc<6>(p, sms, stream);
+#endif
   if (s.K <= 8) return launch_kc<8>(p, sms, stream);
   return launch_kc<16>(p, sms, stream);
 }
