@@ -17,7 +17,11 @@
 // of one row, so each thread owns kU vectors spaced kThreads apart (every
 // warp access is a contiguous 512-byte run).  Blocks stride over tasks,
 // expert-major; the segment range is read once per task.  A thread issues
-// the kU loads of kSU segment rows before adding them, in segment order.  G
+// the kU loads of kSU segment rows before adding them, in segment order.
+// kU = 4, kSU = 1 and a launch bound of 4 blocks per SM (64 registers, 32
+// resident warps) measured best on every workload (1.01-1.09 of the HBM copy
+// peak), against 2 rows in flight with 3 blocks (80 registers: 0.97-1.01),
+// 8 vectors per thread, and 5 or 6 blocks (which spill).  G
 // is read once and home written once, both with streaming (evict-first)
 // accesses.  The segment pointers are read on the device and bounds-checked;
 // nothing is sized from a host copy of the plan.
@@ -42,10 +46,10 @@
 #define MEP_REDUCE_BLOCKS_PER_SM 1024
 #endif
 #ifndef MEP_REDUCE_MIN_BLOCKS
-#define MEP_REDUCE_MIN_BLOCKS 3  // launch bound: resident blocks per SM
+#define MEP_REDUCE_MIN_BLOCKS 4  // launch bound: resident blocks per SM
 #endif
 #ifndef MEP_REDUCE_SEG_UNROLL
-#define MEP_REDUCE_SEG_UNROLL 2  // segment rows in flight per thread
+#define MEP_REDUCE_SEG_UNROLL 1  // segment rows in flight per thread
 #endif
 #ifndef MEP_REDUCE_IMAP
 #define MEP_REDUCE_IMAP 0  // 1: float32 -> binary64 by integer ops (x * 2^-896), one conversion per output
