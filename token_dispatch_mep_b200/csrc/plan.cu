@@ -33,15 +33,21 @@
 //   Phase 3  every block scans T_e over experts (expert offsets); the
 //            coordinator writes maxvio, the offsets, segments, CSR pointers
 //            and replica list; every tile warp walks its ids again in (g, k)
-//            order and gives each pair slot = off_e + tile offset + warp
-//            offset + rank among equal ids earlier in the warp.  The rank
-//            comes from a peer mask (one ballot per id bit; the lanes holding
-//            the same id) and the popcount of the peers below the lane.
-//            This loop bounds phase 3 on large workloads: ~0.9 us per 32-pair
-//            step of the 32 warps, nearly the same with its stores removed
-//            (measured in an instrumented copy), so it is bound by the work
-//            per pair, not by memory; staging src_pair through shared memory
-//            to coalesce its scattered stores was measured slower.
+//            order and gives each pair its position in the expert-sorted
+//            order, off_e + tile offset + warp offset + rank among equal ids
+//            earlier in the warp.  The rank comes from a peer mask (ballots
+//            on the 11 id bits: the lanes holding the same id) and one
+//            population count of the peers below the lane; the last peer
+//            moves the warp's cursor.  The contiguous plan's slot is that
+//            position; the home-first plan maps it through per-expert and
+//            per-rank tables every block derives; the capped plan keeps it in
+//            slot, and after one more grid barrier (while the coordinator,
+//            which built the capped tables meanwhile, writes the segment
+//            table) maps it through the tables the coordinator published.
+//            This loop bounds phase 3 on large workloads (~0.8 us per 32-pair
+//            step of the 32 warps on the Kimi shape); removing its scattered
+//            src_pair stores saved ~2 of its ~11 us (measured in a timing
+//            copy), and staging them through shared memory was slower.
 // A warp whose range exceeds its shared-memory id buffer reads its ids again
 // from global memory (L2 hits) in phase 3.
 #include <atomic>
