@@ -109,6 +109,45 @@ def dram_traffic(name: str, workload: str):
     return None
 
 
+def host_pin_budget(ranks_on_node: int) -> int:
+    """Bytes of pinned host memory one rank may take for the end-to-end
+    inputs: half the node's available memory, shared by its ranks."""
+    import psutil
+    return int(0.5 * psutil.virtual_memory().available / max(1, ranks_on_node))
+
+
+def pinned_sources(tensors: dict, budget: int, pin: bool = True):
+    """Pinned host copies of the device tensors in `tensors` (None entries
+    pass through): whole while they fit `budget` bytes together, otherwise
+    each holds its first rows only, in proportion.  Returns the copies in
+    order and a description of each source."""
+    import torch
+    big = {k: t for k, t in tensors.items() if t is not None}
+    total = sum(t.numel() * t.element_size() for t in big.values())
+    frac = 1.0 if total <= budget else max(budget, 0) / total
+    out, desc = [], {}
+    for k, t in tensors.items():
+        if t is None:
+            out.append(None)
+            continue
+        n = t.shape[0]
+        m = n if frac >= 1.0 else max(1, min(n, int(n * frac)))
+        h = torch.empty((m,) + tuple(t.shape[1:]), dtype=t.dtype, pin_memory=pin).copy_(t[:m])
+        out.append(h)
+        desc[k] = ("pinned whole" if m == n else
+                   f"first {m} of {n} rows pinned, copied {(n + m - 1) // m} times per step")
+    return out[0], out[1], desc
+
+
+def copy_rows(dst, src):
+    """dst[:] = src repeated over dst's rows (host -> device, on the current
+    stream, asynchronous)."""
+    n, m = dst.shape[0], src.shape[0]
+    for r0 in range(0, n, m):
+        r1 = min(n, r0 + m)
+        dst[r0:r1].copy_(src[:r1 - r0], non_blocking=True)
+
+
 # ------------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -554,8 +593,15 @@ def main():
         hi = torch.from_numpy(idx_h).pin_memory()
         hw = torch.from_numpy(w_h).pin_memory()
         hx = torch.empty(x.shape, dtype=x.dtype, **pin).copy_(x)
-        hy = torch.empty(y.shape, dtype=y.dtype, **pin).copy_(y)
-        hG = torch.empty(G.shape, dtype=G.dtype, **pin).copy_(G) if P else None
+        # The large inputs (expert outputs, segment gradients) are pinned whole
+        # when the node's available memory, shared by its ranks, holds them;
+        # otherwise each rank pins their first rows and copies those rows
+        # repeatedly into the device buffer: the same bytes cross PCIe every
+        # step, from a smaller pinned source.
+        local_world = int(os.environ.get("LOCAL_WORLD_SIZE", str(world)))
+        budget = host_pin_budget(local_world) - hx.numel() * hx.element_size()
+        hy, hG, sources = pinned_sources({"y": y, "G": G if P else None}, budget)
+        hG = hG if P else None
         sets = []
         for b in range(2):
             d = dict(idx=idx if b == 0 else torch.empty_like(idx), w=w if b == 0 else torch.empty_like(w),
@@ -571,7 +617,7 @@ def main():
                      hmv=torch.empty(1, dtype=torch.float64, **pin))
             d["ev_in"], d["ev_cmp"], d["ev_out"] = (torch.cuda.Event() for _ in range(3))
             sets.append(d)
-        h2d = sum(t.numel() * t.element_size() for t in (hi, hw, hx, hy) + ((hG,) if P else ()))
+        h2d = sum(t.numel() * t.element_size() for t in (hi, hw, hx, y) + ((G,) if P else ()))
         d2h = sum(t.numel() * t.element_size()
                   for t in (sets[0]["ho"], sets[0]["hsc"], sets[0]["hmv"]) + ((sets[0]["hh"],) if P else ()))
         s_in, s_cmp, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
@@ -584,9 +630,9 @@ def main():
                 d["idx"].copy_(hi, non_blocking=True)
                 d["w"].copy_(hw, non_blocking=True)
                 d["x"].copy_(hx, non_blocking=True)
-                d["y"].copy_(hy, non_blocking=True)
+                copy_rows(d["y"], hy)
                 if P:
-                    d["G"].copy_(hG, non_blocking=True)
+                    copy_rows(d["G"], hG)
                 d["ev_in"].record(s_in)
             with torch.cuda.stream(s_cmp):
                 s_cmp.wait_event(d["ev_in"])
@@ -625,7 +671,8 @@ def main():
             raise RuntimeError("device status not OK after e2e steps")
         e2e = {"value": whole_job_rate(N, world, ms_e2e), "unit": "tokens/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e,
-               "pipeline": "2 buffer sets; H2D, kernels, D2H on 3 streams"}
+               "pipeline": "2 buffer sets; H2D, kernels, D2H on 3 streams",
+               "host_sources": sources}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

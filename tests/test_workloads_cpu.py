@@ -86,3 +86,23 @@ def test_roofline_traffic_follows_the_kernel_source(monkeypatch):
         assert bench.dram_traffic(name, workload) is None                  # kernel changed
     peak, kind = bench.measured_peak()
     assert peak > 1000 and kind in ("measured", "fallback")
+
+
+def test_end_to_end_host_sources_fit_the_budget():
+    """The end-to-end leg pins its large inputs whole when they fit the host
+    budget, else their first rows (in proportion), and the row copy fills
+    every device row from that source."""
+    import torch
+
+    import bench
+    y = torch.arange(40, dtype=torch.float32).reshape(10, 4)
+    G = torch.arange(12, dtype=torch.float32).reshape(6, 2)
+    hy, hG, d = bench.pinned_sources({"y": y, "G": G}, 10 ** 9, pin=False)
+    assert d == {"y": "pinned whole", "G": "pinned whole"} and torch.equal(hy, y) and torch.equal(hG, G)
+    hy, hG, d = bench.pinned_sources({"y": y, "G": None}, 60, pin=False)   # 160 B > 60 B
+    assert hG is None and hy.shape == (3, 4) and torch.equal(hy, y[:3])
+    assert d == {"y": "first 3 of 10 rows pinned, copied 4 times per step"}
+    dst = torch.empty(10, 4)
+    bench.copy_rows(dst, hy)
+    assert torch.equal(dst, y[torch.tensor([0, 1, 2, 0, 1, 2, 0, 1, 2, 0])])
+    assert bench.host_pin_budget(8) > 0
