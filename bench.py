@@ -70,6 +70,8 @@ def parse_args():
                     help="skip the CUDA-graph replay timing of the step")
     ap.add_argument("--no-backward", action="store_true",
                     help="skip the separately timed backward kernels")
+    ap.add_argument("--no-exchange", action="store_true",
+                    help="skip the timing of the per-rank (rank-addressed) exchange calls")
     ap.add_argument("--dispatch-form", choices=["register", "bulk"], default="register",
                     help="dispatch through registers (mep_dispatch) or the bulk-copy engine "
                          "(mep_dispatch_bulk, the staged form kept for comparison)")
@@ -583,6 +585,40 @@ def main():
             raise RuntimeError("device status not OK after the backward kernels")
         del grad_y, grad_w, grad_x
 
+    # ---- the exchange's per-rank calls on this one GPU: rank r dispatches its
+    # own S tokens into the R rank buffers and combines them back from the R
+    # expert-output buffers (here slices of the single buffers, reached
+    # through the rank pointer tables, as peer buffers would be).  All R
+    # ranks' calls run back to back; the bytes are those of the whole calls.
+    exchange = None
+    if not args.no_exchange:
+        SK = S * K
+        btab = mep.rank_pointer_table([buf.view(NK, H)[r * SK:(r + 1) * SK] for r in range(R)], s, H, dev)
+        ytab = mep.rank_pointer_table([y[r * SK:(r + 1) * SK] for r in range(R)], s, H, dev)
+        legs = {"dispatch_ranked_tokens": (lambda: [mep.mep_dispatch_ranked_tokens(
+                    s, H, plan, r * S, x[r * S:(r + 1) * S], btab) for r in range(R)], algo["dispatch"]),
+                "combine_ranked_tokens": (lambda: [mep.mep_combine_ranked_tokens(
+                    s, H, plan, r * S, ytab, w[r * S:(r + 1) * S], out[r * S:(r + 1) * S]) for r in range(R)],
+                    algo["combine"])}
+        exchange = {}
+        for name, (fn, nbytes) in legs.items():
+            ts = []
+            for it in range(3 + 10):
+                flush_l2()
+                b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                b0.record()
+                fn()
+                b1.record()
+                if it >= 3:
+                    ts.append((b0, b1))
+            torch.cuda.synchronize()
+            ms = float(np.median([a.elapsed_time(b) for a, b in ts]))
+            gbs = nbytes / (ms * 1e-3) / 1e9
+            exchange[name] = {"ms_all_ranks": ms, "calls": R, "us_per_rank": ms * 1e3 / R,
+                              "bytes": nbytes, "gbs": gbs, "frac": gbs / peak}
+        if mep.mep_read_status(plan) != 0:
+            raise RuntimeError("device status not OK after the exchange calls")
+
     # ---- e2e: host buffers through the public API, as a user would pipeline
     # it: two device buffer sets, inputs copied host->device on one stream,
     # the path on another, outputs copied back on a third, so the two copy
@@ -700,6 +736,7 @@ def main():
             "gpu_launches": launches_per_step * args.steps,
             "stages_ms": stage_ms,
             "backward_kernels": backward,
+            "exchange_kernels": exchange,
             "graph_replay": graph,
             "home_first_plan": home_first,
             "capped_plan": capped,

@@ -50,7 +50,10 @@
 //
 // Rank-addressed form (mep_combine_ranked): expert outputs are read from R
 // separate rank buffers, slot p being row p % SK of rank_ys[p / SK]; a NULL
-// or misaligned rank pointer is reported, never used.  A token range [g0, g0
+// or misaligned rank pointer is reported, never used.  Each token's K row
+// addresses are resolved once into shared memory and read there by
+// broadcast (resolving them at every step, or holding them in registers,
+// measured 0.77-0.82 of the copy peak against 0.96-1.01 this way).  A token range [g0, g0
 // + N) restricts the kernel to one rank's own tokens (out and w rows are the
 // range's; mep_combine_ranked_tokens).
 //
@@ -215,6 +218,7 @@ template <int KC, bool kRanked>
 __global__ void __launch_bounds__(kThreads, KC == 6 ? MEP_COMBINE_MIN_BLOCKS_K6 : MEP_COMBINE_MIN_BLOCKS)
     combine_row_kernel(CombineParams p) {
   griddep_wait();  // the previous kernel on the stream is complete and visible
+  __shared__ const uint16_t *s_rows[kRanked ? kWarps : 1][kRanked ? KC : 1];  // ranked: the K rows
   constexpr int KG = KC < MEP_COMBINE_GROUP ? KC : MEP_COMBINE_GROUP;
   constexpr int kRU = MEP_COMBINE_ROW_U;
   const int lane = threadIdx.x & 31;
@@ -233,6 +237,18 @@ __global__ void __launch_bounds__(kThreads, KC == 6 ? MEP_COMBINE_MIN_BLOCKS_K6 
     const double wts = (double)wt * kTwo896;  // exact
 #endif
     const unsigned okmask = __ballot_sync(0xffffffffu, sl >= 0);
+    // Ranked form: lane k < K resolves its slot's rank buffer and row once
+    // per token (a division and the pointer checks) into shared memory, which
+    // the warp reads by broadcast at every step (NULL: no row to read).
+    if (kRanked) {
+      __syncwarp();  // the previous token's rows are no longer read
+      if (lane < KC) {
+        bool ok = sl >= 0;
+        const uint16_t *row = ok ? slot_row<true>(p, sl, &ok, &bad) : nullptr;
+        s_rows[threadIdx.x >> 5][lane] = ok ? row : nullptr;
+      }
+      __syncwarp();
+    }
     uint4 *orow = reinterpret_cast<uint4 *>(p.out + g * p.H);
     for (int c0 = 0; c0 < p.chunks; c0 += 32 * kRU) {
       double acc[kRU][8];
@@ -246,9 +262,16 @@ __global__ void __launch_bounds__(kThreads, KC == 6 ? MEP_COMBINE_MIN_BLOCKS_K6 
         uint4 v[KG][kRU];
 #pragma unroll
         for (int j = 0; j < KG; ++j) {
-          const int pk = __shfl_sync(0xffffffffu, sl, kg + j);
-          bool ok = ((okmask >> (kg + j)) & 1) && (unsigned)pk < (unsigned)p.NK;
-          const uint16_t *yrow = slot_row<kRanked>(p, ok ? pk : 0, &ok, &bad);
+          bool ok;
+          const uint16_t *yrow;
+          if (kRanked) {
+            yrow = s_rows[threadIdx.x >> 5][kg + j];
+            ok = yrow != nullptr;
+          } else {
+            const int pk = __shfl_sync(0xffffffffu, sl, kg + j);
+            ok = ((okmask >> (kg + j)) & 1) && (unsigned)pk < (unsigned)p.NK;
+            yrow = slot_row<false>(p, ok ? pk : 0, &ok, &bad);
+          }
 #pragma unroll
           for (int u = 0; u < kRU; ++u) {
             const int c = c0 + u * 32 + lane;
@@ -279,8 +302,14 @@ __global__ void __launch_bounds__(kThreads, KC == 6 ? MEP_COMBINE_MIN_BLOCKS_K6 
           const int pk = __shfl_sync(0xffffffffu, sl, k);
           const double wk = (double)__shfl_sync(0xffffffffu, wt, k);
           bool ok = redo && k < p.K && ((okmask >> k) & 1) && (unsigned)pk < (unsigned)p.NK;
-          bool ignored = false;
-          const uint16_t *yrow = slot_row<kRanked>(p, ok ? pk : 0, &ok, &ignored);
+          const uint16_t *yrow;
+          if (kRanked) {
+            yrow = s_rows[threadIdx.x >> 5][k];
+            ok = ok && yrow != nullptr;
+          } else {
+            bool ignored = false;
+            yrow = slot_row<false>(p, ok ? pk : 0, &ok, &ignored);
+          }
 #pragma unroll
           for (int u = 0; u < kRU; ++u) {
             const int c = c0 + u * 32 + lane;
