@@ -179,27 +179,53 @@ __device__ __forceinline__ const V *seg_row(const ReduceParams &p, const V *G,
 
 // Ranked form: threads t < s1 - s0 resolve segment s0 + t to its row in its
 // rank's buffer.  Returns false if any segment's data was out of range.
+// Ranked form: each segment's place in its rank's slot-ordered list (the
+// row of the rank's gradient buffer that holds it), built once per block
+// from rank_seg_ptr and rank_seg_idx: s_pos[s] = j - rank_seg_ptr[r] for the
+// entry j of rank r listing segment s (r its own rank), -1 for a segment its
+// rank does not list.  (Searching the rank's list for every segment of every
+// task instead measured 0.22-0.77 of the copy peak on the per-home-rank calls.)
+// Every thread of the block calls it.
+__device__ void build_seg_pos(const ReduceParams &p, int *s_pos, int *s_ptr) {
+  const int nrows = p.rows;  // E + R - 1 segment slots
+  for (int i = threadIdx.x; i < nrows; i += blockDim.x) s_pos[i] = -1;
+  for (int r = threadIdx.x; r <= p.R; r += blockDim.x) s_ptr[r] = __ldg(p.rank_seg_ptr + r);
+  __syncthreads();
+  const int total = s_ptr[p.R];
+  if (total >= 0 && total <= nrows) {
+    for (int j = threadIdx.x; j < total; j += blockDim.x) {
+      int lo = 0, hi = p.R;  // the rank r with s_ptr[r] <= j < s_ptr[r + 1]
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (s_ptr[mid] <= j) lo = mid; else hi = mid;
+      }
+      const int sidx = __ldg(p.rank_seg_idx + j);
+      // kept only where the listing rank is the segment's own rank
+      if (sidx >= 0 && sidx < nrows && s_ptr[lo] <= j && __ldg(&p.seg[sidx].y) == lo)
+        s_pos[sidx] = j - s_ptr[lo];
+    }
+  }
+  __syncthreads();
+}
+
+// Ranked form: the rows of segments [s0, s1) into s_rows (NULL where a rank
+// buffer is missing, misaligned or too short, or the segment is not listed
+// by its rank); false if any row is NULL.
 template <typename V>
-__device__ bool resolve_rows(const ReduceParams &p, int s0, int s1, const V **s_rows) {
+__device__ bool resolve_rows(const ReduceParams &p, int s0, int s1, const int *s_pos,
+                             const V **s_rows) {
   bool ok = true;
   for (int t = threadIdx.x; t < s1 - s0; t += blockDim.x) {
     const int s = s0 + t;
     const V *row = nullptr;
     const int r = __ldg(&p.seg[s].y);
-    if (r >= 0 && r < p.R) {
-      const int b = __ldg(p.rank_seg_ptr + r), e = __ldg(p.rank_seg_ptr + r + 1);
-      if (b >= 0 && b <= e && e <= p.rows) {
-        for (int j = b; j < e; ++j)
-          if (__ldg(p.rank_seg_idx + j) == s) {
-            // a rank buffer must be present, aligned to the vector type and
-            // long enough
-            const float *base = p.rank_G[r];
-            if (base != nullptr && (reinterpret_cast<uintptr_t>(base) % sizeof(V)) == 0 &&
-                j - b < p.rank_rows)
-              row = reinterpret_cast<const V *>(base) + (int64_t)(j - b) * p.cols;
-            break;
-          }
-      }
+    const int j = s_pos[s];
+    if (r >= 0 && r < p.R && j >= 0) {
+      // a rank buffer must be present, aligned to the vector type and long
+      // enough
+      const float *base = p.rank_G[r];
+      if (base != nullptr && (reinterpret_cast<uintptr_t>(base) % sizeof(V)) == 0 && j < p.rank_rows)
+        row = reinterpret_cast<const V *>(base) + (int64_t)j * p.cols;
     }
     if (row == nullptr) ok = false;
     s_rows[t] = row;
@@ -211,6 +237,9 @@ template <typename V, bool kRanked>
 __global__ void __launch_bounds__(kThreads, MEP_REDUCE_MIN_BLOCKS) reduce_kernel(ReduceParams p) {
   griddep_wait();  // the previous kernel on the stream is complete and visible
   __shared__ const V *s_rows[kRanked ? kMaxSegPerExpert : 1];
+  __shared__ int s_pos[kRanked ? MEP_MAX_EXPERTS + MEP_MAX_RANKS - 1 : 1];
+  __shared__ int s_ptr[kRanked ? MEP_MAX_RANKS + 1 : 1];
+  if (kRanked) build_seg_pos(p, s_pos, s_ptr);
   const V *G = reinterpret_cast<const V *>(p.G);
   V *home = reinterpret_cast<V *>(p.home);
   const int64_t tile = (int64_t)kThreads * kU;
@@ -228,7 +257,7 @@ __global__ void __launch_bounds__(kThreads, MEP_REDUCE_MIN_BLOCKS) reduce_kernel
     }
     if (kRanked) {
       __syncthreads();  // the previous task's rows are no longer read
-      if (!resolve_rows<V>(p, s0, s1, s_rows)) bad = true;
+      if (!resolve_rows<V>(p, s0, s1, s_pos, s_rows)) bad = true;
       __syncthreads();
     }
     typename Acc<V>::T acc[kU];
@@ -307,8 +336,10 @@ cudaError_t launch(ReduceParams &p, int64_t P, cudaStream_t stream) {
   const int64_t tile = (int64_t)kThreads * kU;
   const int64_t ntask = (int64_t)p.ne * ((p.cols + tile - 1) / tile);
   if (ntask == 0) return cudaSuccess;
-  const int blocks =
-      (int)std::max<int64_t>(1, std::min<int64_t>(ntask, (int64_t)sms * MEP_REDUCE_BLOCKS_PER_SM));
+  // the ranked form builds its segment map once per block: a resident-size
+  // grid, each block striding over many tasks
+  const int64_t cap = kRanked ? (int64_t)sms * MEP_REDUCE_MIN_BLOCKS : (int64_t)sms * MEP_REDUCE_BLOCKS_PER_SM;
+  const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>(ntask, cap));
   if (vec)
     return launch_pdl(reduce_kernel<float4, kRanked>, dim3(blocks), dim3(kThreads), 0, stream, p);
   return launch_pdl(reduce_kernel<float, kRanked>, dim3(blocks), dim3(kThreads), 0, stream, p);
