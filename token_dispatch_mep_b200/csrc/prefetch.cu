@@ -10,6 +10,10 @@
 // grid has a fixed size and strides over num_replicas x tiles tasks; nothing
 // waits for the host.  Replica indices, segment indices and expert ids are
 // range-checked before any address is formed.  Streaming loads and stores.
+// kU = 16 (all 16 loads of a thread in flight before its stores) with a grid
+// cap of 64 blocks per SM measured 0.99-1.02 of the HBM copy peak, against
+// 0.93-0.97 with kU = 4 and 32 blocks per SM (kU = 8, 24 and 32 and caps of
+// 8 to 64 blocks per SM in between).
 #include <algorithm>
 #include <cstdint>
 
@@ -17,7 +21,7 @@
 #include "mep_internal.h"
 
 #ifndef MEP_PREFETCH_BLOCKS_PER_SM
-#define MEP_PREFETCH_BLOCKS_PER_SM 32
+#define MEP_PREFETCH_BLOCKS_PER_SM 64  // grid cap in multiples of the SM count
 #endif
 
 namespace mep {
@@ -25,7 +29,10 @@ namespace mep {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kU = 4;
+#ifndef MEP_PREFETCH_U
+#define MEP_PREFETCH_U 16  // 16-byte vectors per thread per task (all loads in flight together)
+#endif
+constexpr int kU = MEP_PREFETCH_U;
 
 struct PrefetchParams {
   const uint4 *src;
