@@ -179,3 +179,43 @@ def test_missing_rank_buffers_are_reported_not_used():
                                                 mep.pointer_table([g.data_ptr() for g in grads], DEV),
                                                 short, home)
         assert mep.mep_read_status(plan3) == 5
+
+
+FULL = ["r8_e64_h2048", "r16_e256_h7168", "kimi_r64_e896_k16", "skew_r32_zipf1.5"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_per_rank_calls_at_full_size_equal_the_single_buffer_calls(name):
+    """At full size, in the configuration the bench times: every rank's
+    token-range dispatch and combine through the rank pointer tables (rank
+    buffers as slices of the single buffers) equal the single-buffer calls
+    bit for bit, compared on the device (the single-buffer calls are checked
+    against the oracle in test_gpu_parity)."""
+    wl = workloads.WORKLOADS[name]
+    R, S, E, K, H, N, NK = wl.R, wl.S, wl.E, wl.K, wl.H, wl.N, wl.NK
+    SK = S * K
+    s = mep.Shape(R, S, E, K)
+    idx, w = workloads.routing(wl)
+    plan = mep.Plan(s, DEV)
+    mep.mep_plan(s, torch.from_numpy(idx).to(DEV), plan)
+    wd = torch.from_numpy(w).to(DEV)
+    x = workloads.hidden(N, H, seed=1, device=DEV)
+    buf = torch.empty((NK, H), dtype=torch.bfloat16, device=DEV)
+    mep.mep_dispatch(s, H, plan, x, buf)
+    rbuf = torch.full((NK, H), -1, dtype=torch.int16, device=DEV).view(torch.bfloat16)
+    btab = mep.rank_pointer_table([rbuf[r * SK:(r + 1) * SK] for r in range(R)], s, H, DEV)
+    for r in range(R):
+        mep.mep_dispatch_ranked_tokens(s, H, plan, r * S, x[r * S:(r + 1) * S], btab)
+    assert mep.mep_read_status(plan) == 0
+    assert torch.equal(rbuf.view(torch.int16), buf.view(torch.int16))
+    del rbuf, btab, x
+    y = buf  # expert outputs: the dispatched rows (identity experts)
+    out = torch.empty((N, H), dtype=torch.bfloat16, device=DEV)
+    mep.mep_combine(s, H, plan, y, wd, out)
+    rout = torch.full((N, H), -1, dtype=torch.int16, device=DEV).view(torch.bfloat16)
+    ytab = mep.rank_pointer_table([y[r * SK:(r + 1) * SK] for r in range(R)], s, H, DEV)
+    for r in range(R):
+        mep.mep_combine_ranked_tokens(s, H, plan, r * S, ytab, wd[r * S:(r + 1) * S],
+                                      rout[r * S:(r + 1) * S])
+    assert mep.mep_read_status(plan) == 0
+    assert torch.equal(rout.view(torch.int16), out.view(torch.int16))
