@@ -219,3 +219,40 @@ def test_per_rank_calls_at_full_size_equal_the_single_buffer_calls(name):
                                       rout[r * S:(r + 1) * S])
     assert mep.mep_read_status(plan) == 0
     assert torch.equal(rout.view(torch.int16), out.view(torch.int16))
+
+
+@pytest.mark.parametrize("name", ["r8_e64_h2048", "kimi_r64_e896_k16", "skew_r32_adversarial"])
+def test_home_rank_reductions_at_full_size_equal_the_single_buffer_reduce(name):
+    """At full size: every home rank's reduction from per-rank gradient
+    buffers (row j of rank q = q's j-th segment in slot order) equals the
+    single-buffer reduction bit for bit, compared on the device."""
+    wl = workloads.WORKLOADS[name]
+    R, S, E, K, P = wl.R, wl.S, wl.E, wl.K, wl.P
+    s = mep.Shape(R, S, E, K)
+    idx, _ = workloads.routing(wl)
+    plan = mep.Plan(s, DEV)
+    mep.mep_plan(s, torch.from_numpy(idx).to(DEV), plan)
+    G = workloads.seg_grads(wl.seg_rows, P, seed=3, device=DEV)
+    home = torch.empty((E, P), dtype=torch.float32, device=DEV)
+    mep.mep_reduce_replica_grads(s, plan, P, G, home)
+    ph = plan.host()
+    # Each rank buffer holds exactly its own segments' rows (padding all 64
+    # Kimi-shaped buffers to the busiest rank's ~540 rows would not fit one
+    # GPU); the declared length is the largest, and the kernel reads only
+    # rows of segments a rank lists.
+    lists = [ep.local_segments(ph, q) for q in range(R)]
+    rows = max(1, max(len(segs) for segs in lists))
+    grads = []
+    for segs in lists:
+        gq = torch.empty((max(1, len(segs)), P), dtype=torch.float32, device=DEV)
+        for j, (sidx, _, _, _) in enumerate(segs):
+            gq[j] = G[sidx]
+        grads.append(gq)
+    del G
+    gtab = mep.pointer_table([g.data_ptr() for g in grads], DEV)
+    B = E // R
+    rhome = torch.full((E, P), float("nan"), dtype=torch.float32, device=DEV)
+    for q in range(R):
+        mep.mep_reduce_replica_grads_ranked(s, plan, P, q, gtab, rows, rhome[q * B:(q + 1) * B])
+    assert mep.mep_read_status(plan) == 0
+    assert torch.equal(rhome.view(torch.int32), home.view(torch.int32))
