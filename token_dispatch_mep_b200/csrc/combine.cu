@@ -220,6 +220,9 @@ __global__ void __launch_bounds__(kThreads, KC == 6 ? MEP_COMBINE_MIN_BLOCKS_K6 
   griddep_wait();  // the previous kernel on the stream is complete and visible
   __shared__ const uint16_t *s_rows[kRanked ? kWarps : 1][kRanked ? KC : 1];  // ranked: the K rows
   constexpr int KG = KC < MEP_COMBINE_GROUP ? KC : MEP_COMBINE_GROUP;
+  // Groups tile the K terms exactly: a partial last group would read row
+  // pointers past the token's KC entries.
+  static_assert(KC % KG == 0, "load groups must divide the instantiated term count");
   constexpr int kRU = MEP_COMBINE_ROW_U;
   const int lane = threadIdx.x & 31;
   const int64_t nwarps = (int64_t)gridDim.x * kWarps;
