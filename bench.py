@@ -590,18 +590,43 @@ def main():
     # expert-output buffers (here slices of the single buffers, reached
     # through the rank pointer tables, as peer buffers would be).  All R
     # ranks' calls run back to back; the bytes are those of the whole calls.
+    # The whole-range rank-addressed calls (one launch each) are timed beside
+    # them.
     exchange = None
     if not args.no_exchange:
         SK = S * K
         btab = mep.rank_pointer_table([buf.view(NK, H)[r * SK:(r + 1) * SK] for r in range(R)], s, H, dev)
         ytab = mep.rank_pointer_table([y[r * SK:(r + 1) * SK] for r in range(R)], s, H, dev)
         legs = {"dispatch_ranked_tokens": (lambda: [mep.mep_dispatch_ranked_tokens(
-                    s, H, plan, r * S, x[r * S:(r + 1) * S], btab) for r in range(R)], algo["dispatch"]),
+                    s, H, plan, r * S, x[r * S:(r + 1) * S], btab) for r in range(R)], algo["dispatch"], R),
                 "combine_ranked_tokens": (lambda: [mep.mep_combine_ranked_tokens(
                     s, H, plan, r * S, ytab, w[r * S:(r + 1) * S], out[r * S:(r + 1) * S]) for r in range(R)],
-                    algo["combine"])}
+                    algo["combine"], R),
+                # the same kernels over the whole token range in one call each
+                "dispatch_ranked": (lambda: mep.mep_dispatch_ranked(s, H, plan, x, btab), algo["dispatch"], 1),
+                "combine_ranked": (lambda: mep.mep_combine_ranked(s, H, plan, ytab, w, out), algo["combine"], 1)}
+        grads = None
+        if P:
+            # each rank's segment gradients in its own buffer (row j = the
+            # rank's j-th segment in slot order); every home rank reduces its
+            # experts, reading the rows from the buffers that hold them
+            from token_dispatch_mep_b200 import ep
+            ph = plan.host()
+            grads = []
+            for q in range(R):
+                segs = ep.local_segments(ph, q)
+                gq = torch.empty((max(1, len(segs)), P), dtype=torch.float32, device=dev)
+                for j, seg in enumerate(segs):
+                    gq[j] = G[seg[0]]
+                grads.append(gq)
+            rows = max(gq.shape[0] for gq in grads)
+            gtab = mep.pointer_table([gq.data_ptr() for gq in grads], dev)
+            Bx = E // R
+            homes = [home[q * Bx:(q + 1) * Bx] for q in range(R)]
+            legs["reduce_ranked_per_home_rank"] = (lambda: [mep.mep_reduce_replica_grads_ranked(
+                s, plan, P, q, gtab, rows, homes[q]) for q in range(R)], algo["reduce"], R)
         exchange = {}
-        for name, (fn, nbytes) in legs.items():
+        for name, (fn, nbytes, calls) in legs.items():
             ts = []
             for it in range(3 + 10):
                 flush_l2()
@@ -614,10 +639,11 @@ def main():
             torch.cuda.synchronize()
             ms = float(np.median([a.elapsed_time(b) for a, b in ts]))
             gbs = nbytes / (ms * 1e-3) / 1e9
-            exchange[name] = {"ms_all_ranks": ms, "calls": R, "us_per_rank": ms * 1e3 / R,
+            exchange[name] = {"ms_all_ranks": ms, "calls": calls, "us_per_call": ms * 1e3 / calls,
                               "bytes": nbytes, "gbs": gbs, "frac": gbs / peak}
         if mep.mep_read_status(plan) != 0:
             raise RuntimeError("device status not OK after the exchange calls")
+        del grads
 
     # ---- e2e: host buffers through the public API, as a user would pipeline
     # it: two device buffer sets, inputs copied host->device on one stream,
